@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the low-bit routed-expert MoE layer on B200.
+
+Default workload (one JSON line on stdout): the decode stack -- 16 chained
+OLMoE-like MoE FFN layers (hidden 2048, expert intermediate 1024, 64 experts,
+top-8, SwiGLU, W4A16 group-128 experts, bf16 router), no attention, residual
+add between layers, a fresh seeded N(0,1) batch of 8 tokens per step.  One step
+= one pass of the whole hot path (router logits, top-k, permutation, grouped
+gate/up and down GEMV, combine with residual) through all 16 layers, replayed
+as one CUDA graph.  `value` = tokens per second through the 16-layer stack
+(a token counts once per step), whole job over all ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl reference]
+
+Under torchrun each rank runs its own replica on its own seeded batches (the
+layer shards by token, no data-path collective): weak scaling, time = max over
+ranks of the CUDA-event time of the K steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (decode & prefill); weight-stream HBM GB/s vs B200 peak"
+H, I, E, K_TOP, LAYERS = 2048, 1024, 64, 8, 16
+SEED_BASE = 0x5EED0002
+W4_EXPERT_BYTES = (2 * I * H + H * I) // 2 + (2 * I * (H // 128) + H * (I // 128)) * 2  # packed + bf16 scales
+W13_EXPERT_BYTES = 2 * I * H // 2 + 2 * I * (H // 128) * 2
+W2_EXPERT_BYTES = H * I // 2 + H * (I // 128) * 2
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--batch", type=int, default=8)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Largest value over all ranks (every rank takes this collective)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Per-rank stream of step inputs: ranks process disjoint synthetic batches."""
+    return base + 0x10000 * rank
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        time.sleep(0.1)
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        smax = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.5 * smax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def committed_traffic():
+    """DRAM bytes per moe_grouped_ffn call (gate/up + down launches) from the committed
+    ncu summary, with the kernel source hash it was taken on (None if stale/absent)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    p = os.path.join(ROOT, "bit_mixed_precision_router_b200", "csrc", "moe_ffn_gemv.cu")
+    h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------- the GPU arm
+class DecodeStack:
+    """16 chained W4A16 layers on one device, with every buffer a step needs."""
+
+    def __init__(self, moe, torch, device, batch: int, seed: int):
+        self.moe, self.torch, self.dev, self.B = moe, torch, device, batch
+        import synth
+        self.layers = []
+        tmp13 = torch.empty((E, 2 * I, H), dtype=torch.bfloat16, device=device)
+        tmp2 = torch.empty((E, H, I), dtype=torch.bfloat16, device=device)
+        for l in range(LAYERS):
+            ls = seed + 0x100 * (l + 1)
+            wr = torch.empty((E, H), dtype=torch.bfloat16, device=device)
+            moe.moe_synth_normal_bf16(wr, ls + synth.SEED_WR, 0.02)
+            moe.moe_synth_normal_bf16(tmp13, ls + synth.SEED_W13, 0.02)
+            moe.moe_synth_normal_bf16(tmp2, ls + synth.SEED_W2, 0.02)
+            ex = moe.quantize_experts(moe.FMT_W4G128, tmp13, tmp2)
+            self.layers.append((wr, ex))
+        del tmp13, tmp2
+        B = batch
+        self.routing = moe.Routing.empty(B, E, K_TOP, device)
+        self.route_ws = torch.empty(max(moe.moe_route_workspace_bytes(B, E, K_TOP), 16), dtype=torch.uint8,
+                                    device=device)
+        self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(B, H, I, E, K_TOP, moe.FMT_W4G128), 16),
+                                  dtype=torch.uint8, device=device)
+        self.y_rows = torch.empty((B * K_TOP, H), dtype=torch.bfloat16, device=device)
+        self.xs = [torch.empty((B, H), dtype=torch.bfloat16, device=device) for _ in range(LAYERS + 1)]
+        self.n_active = torch.zeros((LAYERS,), dtype=torch.int32, device=device)
+        self.ffn_events = None
+
+    def layer(self, l, log_active=False):
+        moe, wr_ex = self.moe, self.layers[l]
+        wr, ex = wr_ex
+        x, nxt = self.xs[l], self.xs[l + 1]
+        moe.moe_route_topk(x, wr, None, K_TOP, out=self.routing, workspace=self.route_ws)
+        if self.ffn_events is not None:
+            self.ffn_events[l][0].record()
+        moe.moe_grouped_ffn(x, self.routing, ex, I, E, K_TOP, y_rows=self.y_rows, workspace=self.ffn_ws)
+        if self.ffn_events is not None:
+            self.ffn_events[l][1].record()
+        moe.moe_combine(self.y_rows, self.routing, self.B, K_TOP, residual=x, out=nxt)
+        if log_active:
+            self.n_active[l:l + 1].copy_(self.routing.expert_list[:1])
+
+    def step(self, log_active=False):
+        for l in range(LAYERS):
+            self.layer(l, log_active)
+
+    kernels_per_step = LAYERS * 5  # logits, top-k+permute, gate/up, down, combine
+
+
+def run_gpu(args, rank, world, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import bit_mixed_precision_router_b200 as moe
+    moe.load()
+    import synth
+
+    B, K, W = args.batch, args.steps, max(args.warmup, 3)
+    seed = rank_seed(SEED_BASE, rank)
+    stack = DecodeStack(moe, torch, device, B, seed)
+    # a fresh seeded N(0,1) batch for every step (warm-up and timed), resident in HBM
+    n_steps = W + K
+    inputs = torch.empty((n_steps, B, H), dtype=torch.bfloat16, device=device)
+    moe.moe_synth_normal_bf16(inputs, seed + synth.SEED_X, 1.0)
+    torch.cuda.synchronize()
+
+    # eager warm-up (first calls resolve the device symbol before graph capture)
+    for s in range(2):
+        stack.xs[0].copy_(inputs[s])
+        stack.step()
+    torch.cuda.synchronize()
+    moe.moe_check_device_errors()
+
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device)
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            stack.step()
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+
+    for s in range(W):
+        stack.xs[0].copy_(inputs[s])
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for s in range(W, W + K):
+        stack.xs[0].copy_(inputs[s])
+        graph.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_local = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    moe.moe_check_device_errors()
+    ms = max_over_ranks(ms_local, world, device)
+    tokens = B * K * world
+    value = tokens / (ms / 1e3)
+
+    # ---- end-to-end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        host_in = inputs.cpu().pin_memory()
+        host_out = torch.empty((K, B, H), dtype=torch.bfloat16).pin_memory()
+        barrier(world)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for s in range(W, W + K):
+            stack.xs[0].copy_(host_in[s], non_blocking=True)
+            graph.replay()
+            host_out[s - W].copy_(stack.xs[LAYERS], non_blocking=True)
+        t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": B * H * 2,
+               "d2h_bytes_per_step": B * H * 2}
+
+    # ---- roofline of the dominant op: the grouped W4 GEMV (gate/up + down launches of
+    # moe_grouped_ffn), timed with CUDA events recorded on its stream inside a graph
+    stack.ffn_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                        for _ in range(LAYERS)]
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g2, stream=cap):
+            stack.step(log_active=True)
+    torch.cuda.current_stream().wait_stream(cap)
+    ffn_ms, act = [], []
+    n_meas = min(K, 64)
+    for s in range(W, W + n_meas):
+        stack.xs[0].copy_(inputs[s])
+        g2.replay()
+        torch.cuda.synchronize()
+        ffn_ms += [a.elapsed_time(b) for a, b in stack.ffn_events]
+        act += stack.n_active.cpu().tolist()
+    stack.ffn_events = None
+    hbm, bf16_peak, peak_kind = measured_peaks()
+    act_bytes = B * H * 2 + B * K_TOP * I * 2 * 2 + B * K_TOP * H * 2  # x, h (write+read), y_rows
+    algo_bytes = statistics.mean(a * W4_EXPERT_BYTES for a in act) + act_bytes
+    avg_ffn_s = statistics.mean(ffn_ms) / 1e3
+    achieved = algo_bytes / avg_ffn_s / 1e9
+    traffic = committed_traffic()
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_kind": peak_kind,
+                "traffic": traffic["dram_bytes_per_call"] if traffic else None,
+                "kernel": "k_ffn_gemv<W4> gate/up + down (one moe_grouped_ffn call)",
+                "algorithmic_bytes_per_call": round(algo_bytes), "avg_call_us": round(avg_ffn_s * 1e6, 2),
+                "distinct_experts_per_layer": round(statistics.mean(act), 2)}
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, "
+                                                          "N(0,0.02) bf16 weights quantised to W4A16 g128)",
+            "config": {"workload": "decode stack: 16 chained OLMoE-like MoE FFN layers (H2048 I1024 E64 top-8, "
+                                   "W4A16 g128 experts, bf16 router), residual add, batch %d tokens/step" % B,
+                       "layers": LAYERS, "batch": B, "hidden": H, "intermediate": I, "experts": E, "top_k": K_TOP,
+                       "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "no flush: each step streams ~%.1f GB of distinct expert weights, > 126 MB L2"
+                             % (statistics.mean(act) * W4_EXPERT_BYTES * LAYERS / 1e9)},
+            "gpu_launches": stack.kernels_per_step * K,
+            "clocks": clk, "roofline": roofline, "e2e": e2e,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        del graph, g2
+        dist.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------------- the oracle (CPU) arm
+def oracle_sample(batch: int, layers_timed: int, seed: int):
+    """Times the CPU oracle on a bounded sample of the decode stack: `layers_timed`
+    consecutive layers of one step (weights prepared untimed).  Returns
+    (tokens/s through the 16-layer stack, seconds timed, threads used)."""
+    import numpy as np
+
+    import synth
+    from oracle.ffn import FMT_W4G128, Experts, stack_layer_step
+    from oracle.quant import quantize_w4g128
+    from oracle.routing import router_logits, topk_softmax
+    x = synth.normal_bf16(seed + synth.SEED_X, batch * H, 1.0).reshape(batch, H)
+    timed = 0.0
+    for l in range(layers_timed):
+        ls = seed + 0x100 * (l + 1)
+        wr = synth.normal_bf16(ls + synth.SEED_WR, E * H, 0.02).reshape(E, H)
+        ids, _ = topk_softmax(router_logits(x, wr), K_TOP)
+        # quantise only the experts this layer routes to (offline work, untimed)
+        w13q = np.zeros((E, 2 * I, H // 8), np.uint32)
+        w13s = np.zeros((E, 2 * I, H // 128), np.uint16)
+        w2q = np.zeros((E, H, I // 8), np.uint32)
+        w2s = np.zeros((E, H, I // 128), np.uint16)
+        for e in sorted(set(ids.reshape(-1).tolist())):
+            a = quantize_w4g128(synth.normal_rows_bf16(ls + synth.SEED_W13, (2 * I, H), 0.02, e, 1))
+            b = quantize_w4g128(synth.normal_rows_bf16(ls + synth.SEED_W2, (H, I), 0.02, e, 1))
+            w13q[e], w13s[e], w2q[e], w2s[e] = a[0][0], a[1][0], b[0][0], b[1][0]
+        ex = Experts(FMT_W4G128, w13q, w13s, w2q, w2s)
+        t0 = time.perf_counter()
+        x, _ = stack_layer_step(x, wr, ex, K_TOP)
+        timed += time.perf_counter() - t0
+    per_step = timed * LAYERS / layers_timed
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    return batch / per_step, timed, threads
+
+
+def cpu_baseline(batch: int, seed: int):
+    layers_timed = 2
+    v, secs, thr = oracle_sample(batch, layers_timed, seed)
+    return {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{layers_timed} of the 16 layers of one decode step at batch {batch} "
+                      f"({secs:.1f} s of CPU work), scaled to the full step"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on this workload's config."""
+    if rank != 0:
+        return None
+    B = args.batch
+    K, W = args.steps, args.warmup
+    # each step: a bounded sample (2 layers of the stack), W + K of them kept short
+    n = max(1, min(K, 3))
+    vals = []
+    for s in range(n):
+        v, secs, thr = oracle_sample(B, 2, SEED_BASE + s)
+        vals.append(v)
+    value = statistics.mean(vals)
+    return {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(B / value * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "decode stack: 16 chained OLMoE-like MoE FFN layers (H2048 I1024 E64 top-8, "
+                                   "W4A16 g128 experts, bf16 router), residual add, batch %d tokens/step" % B,
+                       "layers": LAYERS, "batch": B},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                             "sample": f"{n} sampled steps, each 2 of the 16 layers of a decode step, "
+                                       f"scaled to the full step"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    res = run_gpu(args, rank, world, local)
+    if rank == 0 and res is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args.batch, SEED_BASE)
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,277 @@
+"""Python binding of libmoe.so, the C ABI of the low-bit routed-expert MoE FFN
+layer (include/moe.h, include/moe_synth.h).
+
+Argument marshalling only: each function takes torch CUDA tensors, passes their
+device pointers and the current CUDA stream to the C entry point of the same
+name, and raises MoeError on a non-zero status.  Every computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing the
+binding without the built library raises at ``load()``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+FMT_W4G128, FMT_BITPLANE8, FMT_NVFP4 = 0, 1, 2
+MAX_EXPERTS, MAX_TOPK = 1024, 32
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_MISALIGNED", 6: "MOE_ERR_DEVICE_TIMEOUT"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+class RoutingT(ctypes.Structure):
+    _fields_ = [("topk_ids", ctypes.c_void_p), ("topk_w", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
+                ("sorted_pair", ctypes.c_void_p), ("pair_to_row", ctypes.c_void_p),
+                ("expert_list", ctypes.c_void_p)]
+
+
+class ExpertsT(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int), ("w13", ctypes.c_void_p), ("w13_scale", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p), ("w13_gscale", ctypes.c_void_p),
+                ("w2_gscale", ctypes.c_void_p)]
+
+
+_lib = None
+_vp, _i64, _sz, _u64, _d = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_double
+
+_SIGS = {
+    "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "moe_abi_version": ([], ctypes.c_int),
+    "moe_quantize_w4g128": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], ctypes.c_int),
+    "moe_pack_bitplanes": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], ctypes.c_int),
+    "moe_quantize_nvfp4": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moe_route_workspace_bytes": ([_i64, _i64, _i64], _sz),
+    "moe_route_topk": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.POINTER(RoutingT), _vp, _sz, _vp],
+                       ctypes.c_int),
+    "moe_select_bits": ([_vp, _i64, _i64, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_uint8), _vp,
+                         _vp], ctypes.c_int),
+    "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
+    "moe_grouped_ffn": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
+                         _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_combine": ([_vp, ctypes.POINTER(RoutingT), _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
+    "moe_check_device_errors": ([_vp], ctypes.c_int),
+    "moe_synth_normal_bf16": ([_vp, _i64, _i64, _u64, _d, _vp], ctypes.c_int),
+    "moe_synth_uniform_bf16": ([_vp, _i64, _i64, _u64, _d, _d, _vp], ctypes.c_int),
+}
+
+
+def load(path: str = LIB_PATH):
+    """Load libmoe.so (built by ``python -m bit_mixed_precision_router_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m bit_mixed_precision_router_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (args, res) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGS)
+
+
+def _call(name: str, *args) -> None:
+    st = getattr(load(), name)(*args)
+    if st != 0:
+        raise MoeError(name, st)
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _p(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    """bf16 tensors travel as their 16-bit patterns."""
+    if t.dtype == torch.bfloat16:
+        return t
+    if t.dtype in (torch.int16, torch.uint16):
+        return t
+    raise TypeError(f"expected bf16 data, got {t.dtype}")
+
+
+# ---------------------------------------------------------------- offline quantisers
+def moe_quantize_w4g128(w: torch.Tensor, packed: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                        stream=None):
+    """bf16 [E][N][K] -> (packed int32 [E][N][K/8] holding uint32 words, scales bf16 [E][N][K/128])."""
+    E, N, K = w.shape
+    packed = torch.empty((E, N, K // 8), dtype=torch.int32, device=w.device) if packed is None else packed
+    scales = torch.empty((E, N, K // 128), dtype=torch.bfloat16, device=w.device) if scales is None else scales
+    _call("moe_quantize_w4g128", _p(_bits(w)), E, N, K, _p(packed), _p(scales), _stream(stream))
+    return packed, scales
+
+
+def moe_pack_bitplanes(w: torch.Tensor, planes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                       stream=None):
+    """bf16 [E][N][K] -> (planes int32 [E][8][N][K/32], scales bf16 [E][N][K/128])."""
+    E, N, K = w.shape
+    planes = torch.empty((E, 8, N, K // 32), dtype=torch.int32, device=w.device) if planes is None else planes
+    scales = torch.empty((E, N, K // 128), dtype=torch.bfloat16, device=w.device) if scales is None else scales
+    _call("moe_pack_bitplanes", _p(_bits(w)), E, N, K, _p(planes), _p(scales), _stream(stream))
+    return planes, scales
+
+
+def moe_quantize_nvfp4(w: torch.Tensor, codes=None, block_scales=None, gscale=None, stream=None):
+    """bf16 [E][N][K] -> (codes uint8 [E][N][K/2], block_scales uint8 [E][N][K/16], gscale fp32 [E])."""
+    E, N, K = w.shape
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device) if codes is None else codes
+    block_scales = (torch.empty((E, N, K // 16), dtype=torch.uint8, device=w.device)
+                    if block_scales is None else block_scales)
+    gscale = torch.empty((E,), dtype=torch.float32, device=w.device) if gscale is None else gscale
+    _call("moe_quantize_nvfp4", _p(_bits(w)), E, N, K, _p(codes), _p(block_scales), _p(gscale), _stream(stream))
+    return codes, block_scales, gscale
+
+
+# ---------------------------------------------------------------- routing
+@dataclass
+class Routing:
+    """Device buffers of one routing (moe_routing_t)."""
+    topk_ids: torch.Tensor
+    topk_w: torch.Tensor
+    expert_offsets: torch.Tensor
+    sorted_pair: torch.Tensor
+    pair_to_row: torch.Tensor
+    expert_list: torch.Tensor
+
+    @staticmethod
+    def empty(T: int, E: int, k: int, device="cuda") -> "Routing":
+        P = max(T * k, 1)
+        i32 = dict(dtype=torch.int32, device=device)
+        return Routing(torch.empty(P, **i32), torch.empty(P, dtype=torch.float32, device=device),
+                       torch.empty(E + 1, **i32), torch.empty(P, **i32), torch.empty(P, **i32),
+                       torch.empty(E + 1, **i32))
+
+    def c(self) -> RoutingT:
+        return RoutingT(_p(self.topk_ids), _p(self.topk_w), _p(self.expert_offsets), _p(self.sorted_pair),
+                        _p(self.pair_to_row), _p(self.expert_list))
+
+
+def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:
+    return int(load().moe_route_workspace_bytes(T, E, k))
+
+
+def moe_route_topk(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None, k: int,
+                   out: Routing | None = None, workspace: torch.Tensor | None = None, stream=None) -> Routing:
+    T, H = x.shape
+    E = w_router.shape[0]
+    out = Routing.empty(T, E, k, x.device) if out is None else out
+    need = moe_route_workspace_bytes(T, E, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    rc = out.c()
+    _call("moe_route_topk", _p(_bits(x)), _p(_bits(w_router)), _p(bias), T, H, E, k, ctypes.byref(rc),
+          _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return out
+
+
+def moe_select_bits(topk_w: torch.Tensor, k: int, thresholds=(0.05, 0.15, 0.30), choices=(2, 3, 4, 8),
+                    bits: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    n = topk_w.numel()
+    T = n // k
+    bits = torch.empty(max(n, 1), dtype=torch.uint8, device=topk_w.device) if bits is None else bits
+    thr = (ctypes.c_float * 3)(*thresholds)
+    ch = (ctypes.c_uint8 * 4)(*choices)
+    _call("moe_select_bits", _p(topk_w), T, k, thr, ch, _p(bits), _stream(stream))
+    return bits
+
+
+# ---------------------------------------------------------------- FFN and combine
+@dataclass
+class Experts:
+    """Device buffers of quantised experts (moe_experts_t)."""
+    fmt: int
+    w13: torch.Tensor
+    w13_scale: torch.Tensor
+    w2: torch.Tensor
+    w2_scale: torch.Tensor
+    w13_gscale: torch.Tensor | None = None
+    w2_gscale: torch.Tensor | None = None
+
+    def c(self) -> ExpertsT:
+        return ExpertsT(self.fmt, _p(self.w13), _p(self.w13_scale), _p(self.w2), _p(self.w2_scale),
+                        _p(self.w13_gscale), _p(self.w2_gscale))
+
+
+def quantize_experts(fmt: int, w13: torch.Tensor, w2: torch.Tensor, stream=None) -> Experts:
+    """Quantise bf16 w13 [E][2I][H] and w2 [E][H][I] into one of the three formats."""
+    if fmt == FMT_W4G128:
+        a, b = moe_quantize_w4g128(w13, stream=stream), moe_quantize_w4g128(w2, stream=stream)
+        return Experts(fmt, a[0], a[1], b[0], b[1])
+    if fmt == FMT_BITPLANE8:
+        a, b = moe_pack_bitplanes(w13, stream=stream), moe_pack_bitplanes(w2, stream=stream)
+        return Experts(fmt, a[0], a[1], b[0], b[1])
+    if fmt == FMT_NVFP4:
+        a, b = moe_quantize_nvfp4(w13, stream=stream), moe_quantize_nvfp4(w2, stream=stream)
+        return Experts(fmt, a[0], a[1], b[0], b[1], a[2], b[2])
+    raise ValueError(fmt)
+
+
+def moe_ffn_workspace_bytes(T: int, H: int, I: int, E: int, k: int, fmt: int) -> int:
+    return int(load().moe_ffn_workspace_bytes(T, H, I, E, k, fmt))
+
+
+def moe_grouped_ffn(x: torch.Tensor, routing: Routing, experts: Experts, I: int, E: int, k: int,
+                    bits: torch.Tensor | None = None, y_rows: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    T, H = x.shape
+    y_rows = torch.empty((max(T * k, 1), H), dtype=torch.bfloat16, device=x.device) if y_rows is None else y_rows
+    need = moe_ffn_workspace_bytes(T, H, I, E, k, experts.fmt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    rc, ec = routing.c(), experts.c()
+    _call("moe_grouped_ffn", _p(_bits(x)), ctypes.byref(rc), ctypes.byref(ec), _p(bits), T, H, I, E, k,
+          _p(y_rows), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return y_rows
+
+
+def moe_combine(y_rows: torch.Tensor, routing: Routing, T: int, k: int, residual: torch.Tensor | None = None,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    H = y_rows.shape[1]
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=y_rows.device) if out is None else out
+    rc = routing.c()
+    _call("moe_combine", _p(y_rows), ctypes.byref(rc), _p(residual), T, H, k, _p(out), _stream(stream))
+    return out
+
+
+def moe_check_device_errors(stream=None) -> None:
+    _call("moe_check_device_errors", _stream(stream))
+
+
+# ---------------------------------------------------------------- synthetic inputs
+def moe_synth_normal_bf16(out: torch.Tensor, seed: int, std: float, start: int = 0, stream=None) -> torch.Tensor:
+    _call("moe_synth_normal_bf16", _p(out), out.numel(), start, seed & (2 ** 64 - 1), float(std), _stream(stream))
+    return out
+
+
+def moe_synth_uniform_bf16(out: torch.Tensor, seed: int, lo: float, hi: float, start: int = 0,
+                           stream=None) -> torch.Tensor:
+    _call("moe_synth_uniform_bf16", _p(out), out.numel(), start, seed & (2 ** 64 - 1), float(lo), float(hi),
+          _stream(stream))
+    return out

@@ -1,0 +1,230 @@
+// The C ABI (moe.h, moe_synth.h): host-side argument validation, then dispatch to
+// the launchers.  Nothing here allocates device memory or synchronises, except
+// moe_check_device_errors.
+#include <stdint.h>
+
+#include <climits>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+#include "moe_synth.h"
+
+// The device error word (one per device, bit kErrWaitTimeout set by a kernel
+// whose bounded wait ran out).
+__device__ unsigned g_moe_error_word;
+
+namespace moe {
+
+unsigned* device_error_word() {
+  static unsigned* cached[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_error_word) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<unsigned*>(p);
+  }
+  return cached[dev];
+}
+
+}  // namespace moe
+
+namespace {
+
+constexpr size_t kMaxDynSmem = 220 * 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
+
+moe_status_t check_quant_args(const void* w, int64_t E, int64_t N, int64_t K, const void* o1, const void* o2,
+                              int64_t kmult) {
+  if (!w || !o1 || !o2) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || N < 1 || K < 1) return MOE_ERR_INVALID_ARG;
+  if (K % kmult != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (E > INT_MAX || N > INT_MAX || E * N > (int64_t(1) << 40) / K) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(w) || !aligned16(o1) || !aligned16(o2)) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+moe_status_t check_routing(const moe_routing_t* r) {
+  if (!r) return MOE_ERR_INVALID_ARG;
+  const void* ps[] = {r->topk_ids, r->topk_w, r->expert_offsets, r->sorted_pair, r->pair_to_row, r->expert_list};
+  for (const void* p : ps)
+    if (!p) return MOE_ERR_INVALID_ARG;
+  for (const void* p : ps)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+moe_status_t check_route_shape(int64_t T, int64_t E, int64_t k) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (k < 1 || k > E || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT_MAX / k) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+size_t ffn_smem_need(int64_t K, moe_format_t fmt) {
+  // padded rows as laid out by the FFN kernels (16 rows; 8 planes for bitplanes)
+  if (fmt == MOE_FMT_BITPLANE8) return size_t(8 * 16) * size_t(K / 8 + 16);
+  return size_t(16) * size_t(K / 2 + 64);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+  }
+  return "unknown status";
+}
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+moe_status_t moe_quantize_w4g128(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint32_t* packed,
+                                 uint16_t* scales, moe_stream_t stream) {
+  moe_status_t s = check_quant_args(w, E, N, K, packed, scales, 128);
+  if (s != MOE_OK) return s;
+  return from_cuda(moe::launch_quantize_w4g128(w, E, N, K, packed, scales, as_stream(stream)));
+}
+
+moe_status_t moe_pack_bitplanes(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint32_t* planes,
+                                uint16_t* scales, moe_stream_t stream) {
+  moe_status_t s = check_quant_args(w, E, N, K, planes, scales, 128);
+  if (s != MOE_OK) return s;
+  return from_cuda(moe::launch_pack_bitplanes(w, E, N, K, planes, scales, as_stream(stream)));
+}
+
+moe_status_t moe_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* codes,
+                                uint8_t* block_scales, float* gscale, moe_stream_t stream) {
+  moe_status_t s = check_quant_args(w, E, N, K, codes, block_scales, 32);
+  if (s != MOE_OK) return s;
+  if (!gscale) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(gscale)) return MOE_ERR_MISALIGNED;
+  if (E > 65535) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(moe::launch_quantize_nvfp4(w, E, N, K, codes, block_scales, gscale, as_stream(stream)));
+}
+
+size_t moe_route_workspace_bytes(int64_t T, int64_t E, int64_t k) {
+  if (T < 0 || E < 1 || k < 1) return 0;
+  return moe::route_workspace_bytes(T, E, k);
+}
+
+moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const float* bias, int64_t T, int64_t H,
+                            int64_t E, int64_t k, const moe_routing_t* out, void* workspace,
+                            size_t workspace_bytes, moe_stream_t stream) {
+  moe_status_t s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  if (H < 256 || H % 256 != 0 || H > INT_MAX / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;  // nothing to route; no pointer is read
+  if (!x || !w_router) return MOE_ERR_INVALID_ARG;
+  if ((s = check_routing(out)) != MOE_OK) return s;
+  if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned16(bias))) return MOE_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < moe::route_workspace_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_route(x, w_router, bias, int(T), int(H), int(E), int(k), *out, workspace,
+                                     as_stream(stream)));
+}
+
+moe_status_t moe_select_bits(const float* topk_w, int64_t T, int64_t k, const float thresholds[3],
+                             const uint8_t choices[4], uint8_t* bits, moe_stream_t stream) {
+  if (!topk_w || !thresholds || !choices || !bits) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+  if (!(thresholds[0] <= thresholds[1] && thresholds[1] <= thresholds[2])) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (choices[i] < 1 || choices[i] > 8) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_w) || !aligned16(bits)) return MOE_ERR_MISALIGNED;
+  if (T == 0) return MOE_OK;
+  return from_cuda(moe::launch_select_bits(topk_w, T * k, thresholds, choices, bits, as_stream(stream)));
+}
+
+size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, moe_format_t fmt) {
+  if (T < 0 || H < 1 || I < 1 || k < 1) return 0;
+  return moe::ffn_workspace_bytes(T, H, I, E, k, fmt);
+}
+
+moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing, const moe_experts_t* experts,
+                             const uint8_t* bits, int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                             uint16_t* y_rows, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  if (!experts) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  const moe_experts_t& ex = *experts;
+  if (ex.fmt != MOE_FMT_W4G128 && ex.fmt != MOE_FMT_BITPLANE8 && ex.fmt != MOE_FMT_NVFP4)
+    return MOE_ERR_INVALID_ARG;
+  if (!ex.w13 || !ex.w13_scale || !ex.w2 || !ex.w2_scale) return MOE_ERR_INVALID_ARG;
+  if (ex.fmt == MOE_FMT_NVFP4 && (!ex.w13_gscale || !ex.w2_gscale)) return MOE_ERR_INVALID_ARG;
+  if (H < 256 || H % 256 != 0 || I < 128 || I % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (ffn_smem_need(H, ex.fmt) > kMaxDynSmem || ffn_smem_need(I, ex.fmt) > kMaxDynSmem)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (int64_t(E) * 2 * I > INT_MAX || T * k > INT_MAX / (H > I ? H : I)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;  // no pairs; no activation or output pointer is read
+  if (!x || !y_rows) return MOE_ERR_INVALID_ARG;
+  if (ex.fmt == MOE_FMT_BITPLANE8 && !bits) return MOE_ERR_INVALID_ARG;
+  if ((s = check_routing(routing)) != MOE_OK) return s;
+  const void* ps[] = {x, ex.w13, ex.w13_scale, ex.w2, ex.w2_scale, y_rows};
+  for (const void* p : ps)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  if ((bits && !aligned16(bits)) || (ex.w13_gscale && !aligned16(ex.w13_gscale)) ||
+      (ex.w2_gscale && !aligned16(ex.w2_gscale)))
+    return MOE_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < moe::ffn_workspace_bytes(T, H, I, E, k, ex.fmt)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MOE_ERR_MISALIGNED;
+  if (!moe::device_error_word()) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_grouped_ffn(x, *routing, ex, bits, int(T), int(H), int(I), int(E), int(k), y_rows,
+                                           workspace, as_stream(stream)));
+}
+
+moe_status_t moe_combine(const uint16_t* y_rows, const moe_routing_t* routing, const uint16_t* residual,
+                         int64_t T, int64_t H, int64_t k, uint16_t* out, moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > MOE_MAX_TOPK || H < 8) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT_MAX / k || T * k > INT64_MAX / H) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;  // no tokens; no pointer is read
+  if (!y_rows || !out) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = check_routing(routing);
+  if (s != MOE_OK) return s;
+  if (!aligned16(y_rows) || !aligned16(out) || (residual && !aligned16(residual))) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_combine(y_rows, *routing, residual, int(T), int(H), int(k), out, as_stream(stream)));
+}
+
+moe_status_t moe_check_device_errors(moe_stream_t stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_moe_error_word, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_moe_error_word, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_DEVICE_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_synth_normal_bf16(uint16_t* out, int64_t n, int64_t start, uint64_t seed, double stddev,
+                                   moe_stream_t stream) {
+  if (!out || n < 0 || start < 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (n / 256 >= int64_t(INT_MAX)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(moe::launch_synth_normal(out, n, start, seed, stddev, as_stream(stream)));
+}
+
+moe_status_t moe_synth_uniform_bf16(uint16_t* out, int64_t n, int64_t start, uint64_t seed, double lo, double hi,
+                                    moe_stream_t stream) {
+  if (!out || n < 0 || start < 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (n / 256 >= int64_t(INT_MAX)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(moe::launch_synth_uniform(out, n, start, seed, lo, hi, as_stream(stream)));
+}
+
+}  // extern "C"

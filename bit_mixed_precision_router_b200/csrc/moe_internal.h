@@ -1,0 +1,40 @@
+// Host-side launchers behind the C ABI (moe_api.cu).  Arguments are validated by
+// the caller; each launcher only enqueues kernels and returns cudaGetLastError().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+cudaError_t launch_quantize_w4g128(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint32_t* packed,
+                                   uint16_t* scales, cudaStream_t st);
+cudaError_t launch_pack_bitplanes(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint32_t* planes,
+                                  uint16_t* scales, cudaStream_t st);
+cudaError_t launch_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* codes,
+                                  uint8_t* block_scales, float* gscale, cudaStream_t st);
+
+// Routing: logits into `logits` (fp32 [T][E]), then top-k and the permutation.
+size_t route_workspace_bytes(int64_t T, int64_t E, int64_t k);
+cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                         const moe_routing_t& out, void* ws, cudaStream_t st);
+cudaError_t launch_select_bits(const float* w, int64_t n, const float thr[3], const uint8_t ch[4],
+                               uint8_t* bits, cudaStream_t st);
+
+// Grouped FFN.
+size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, moe_format_t fmt);
+cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
+                               const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,
+                               void* ws, cudaStream_t st);
+
+cudaError_t launch_combine(const uint16_t* y_rows, const moe_routing_t& r, const uint16_t* residual, int T,
+                           int H, int k, uint16_t* out, cudaStream_t st);
+
+cudaError_t launch_synth_normal(uint16_t* out, int64_t n, int64_t start, uint64_t seed, double stddev,
+                                cudaStream_t st);
+cudaError_t launch_synth_uniform(uint16_t* out, int64_t n, int64_t start, uint64_t seed, double lo, double hi,
+                                 cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,227 @@
+/*
+ * moe.h -- C ABI of the low-bit routed-expert MoE FFN layer for NVIDIA B200 (sm_100a).
+ *
+ * One Mixture-of-Experts feed-forward layer whose routed experts hold low-bit
+ * weights, run as: router logits -> top-k with softmax weights -> permutation of
+ * the (token, slot) pairs by expert -> grouped SwiGLU expert GEMV/GEMM that
+ * dequantises the weights in-kernel -> routing-weighted combine.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [ExactMoE]  "Every Expert Counts: ExactMoE for Memory-Efficient W4A16
+ *               Inference", abstract: symmetric group-128 four-bit weights on the
+ *               routed experts only, router kept in BF16, top-k unchanged, all
+ *               selected experts executed by fused grouped kernels.
+ *   [PagedMoE]  "PagedMoE: Cross-Precision Expert Caching for Token-Level Dynamic
+ *               Precision in SSD-Resident MoE Inference", abstract: one stored
+ *               expert state in a bitplane layout, lower precisions being
+ *               prefixes of higher ones; prefix length chosen per token from the
+ *               routing weights; prefixes executed directly.
+ *   [MatMoE]    "MatMoE: Matryoshka Mixture-of-Experts with Dynamic Mixed-Precision
+ *               Quantization for Efficient Inference", abstract: floor-and-
+ *               compensation quantisation; bit-width per expert from routing scores.
+ *   [MoET]      "MoET in FP4 MoE Inference" (Q&A page), answer and references:
+ *               FP4/INT4 expert weights, router at higher precision, NVFP4.
+ *
+ * Conventions shared by every entry point
+ *   - bf16 values are passed as uint16_t bit patterns.
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise, owned
+ *     by the caller; the library never allocates, frees or keeps a pointer after
+ *     the call returns.  Device pointers must be 16-byte aligned.
+ *   - Every call only enqueues work on `stream` (a cudaStream_t; NULL means the
+ *     legacy default stream) and returns without synchronising.
+ *   - All arguments are validated on the host before anything is launched; an
+ *     invalid call launches nothing and returns an error code.  A failed launch
+ *     returns MOE_ERR_CUDA.  No C++ exception crosses the ABI.
+ *   - T = 0 (no tokens) is valid and launches nothing.
+ *   - Shapes: weights are row-major [E][N][K] with K contiguous.  The gate/up
+ *     matrix w13 of expert e is [2I][H] (rows 0..I-1 gate, I..2I-1 up); the down
+ *     matrix w2 is [H][I].
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+/* Size limits enforced by validation. */
+#define MOE_MAX_EXPERTS 1024 /* E */
+#define MOE_MAX_TOPK 32      /* k */
+
+typedef void* moe_stream_t; /* cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside the limits stated per call */
+  MOE_ERR_WORKSPACE = 3,         /* workspace pointer null or smaller than required */
+  MOE_ERR_CUDA = 4,              /* a CUDA launch or runtime call failed */
+  MOE_ERR_MISALIGNED = 5,        /* a device pointer is not 16-byte aligned */
+  MOE_ERR_DEVICE_TIMEOUT = 6     /* a kernel gave up waiting (see moe_check_device_errors) */
+} moe_status_t;
+
+typedef enum {
+  MOE_FMT_W4G128 = 0,   /* INT4, symmetric, one bf16 scale per 128 K-elements [ExactMoE] */
+  MOE_FMT_BITPLANE8 = 1,/* 8-bit symmetric codes stored as 8 bitplanes [PagedMoE], read at b planes */
+  MOE_FMT_NVFP4 = 2     /* E2M1 + E4M3 scale per 16 + fp32 scale per expert matrix [MoET] */
+} moe_format_t;
+
+/* Routing of T tokens to k experts each; every array is device memory.
+ * Pair p = t*k + j is token t's j-th choice. */
+typedef struct {
+  int32_t* topk_ids;       /* [T*k]  expert of pair p; slots ordered by logit descending, ties by lower id */
+  float* topk_w;           /* [T*k]  routing weight of pair p (softmax over the token's k logits) */
+  int32_t* expert_offsets; /* [E+1]  pairs routed to experts < e; offsets[E] = T*k */
+  int32_t* sorted_pair;    /* [T*k]  pair held by sorted row r; ascending p inside each expert */
+  int32_t* pair_to_row;    /* [T*k]  inverse of sorted_pair */
+  int32_t* expert_list;    /* [E+1]  [0] = number A of experts with >= 1 pair, [1..A] their ids ascending */
+} moe_routing_t;
+
+/* Quantised expert weights (device memory), as written by the quantisers below.
+ *   W4G128:    w13 uint32 [E][2I][H/8],  w13_scale bf16 [E][2I][H/128];
+ *              w2  uint32 [E][H][I/8],   w2_scale  bf16 [E][H][I/128].
+ *   BITPLANE8: w13 uint32 [E][8][2I][H/32], w13_scale bf16 [E][2I][H/128];
+ *              w2  uint32 [E][8][H][I/32],  w2_scale  bf16 [E][H][I/128].
+ *   NVFP4:     w13 uint8 [E][2I][H/2], w13_scale E4M3 uint8 [E][2I][H/16], w13_gscale fp32 [E];
+ *              w2  uint8 [E][H][I/2],  w2_scale  E4M3 uint8 [E][H][I/16],  w2_gscale  fp32 [E]. */
+typedef struct {
+  moe_format_t fmt;
+  const void* w13;
+  const void* w13_scale;
+  const void* w2;
+  const void* w2_scale;
+  const float* w13_gscale; /* NVFP4 only, else NULL */
+  const float* w2_gscale;  /* NVFP4 only, else NULL */
+} moe_experts_t;
+
+/* Static string for a status code (never NULL). */
+const char* moe_status_string(moe_status_t status);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int moe_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Offline weight preparation (not part of a layer step).
+ * ------------------------------------------------------------------------ */
+
+/* INT4 symmetric group-128 quantisation [ExactMoE].
+ * Per row and per group of 128 consecutive K elements: scale = bf16(max|w| / 7)
+ * (fp32 division, round to nearest even); q = clamp(rint(w / scale), -8, 7)
+ * (fp32 division, ties to even); an all-zero group has scale 0 and q = 0.
+ * Storage: u = q + 8, element k of a row in bits 4*(k%8).. of uint32 word k/8.
+ *   w      bf16 [E][N][K];  packed uint32 [E][N][K/8];  scales bf16 [E][N][K/128].
+ * Requires E, N >= 1, K >= 128, K % 128 == 0.  Bit-exact (integer decisions in IEEE fp32). */
+moe_status_t moe_quantize_w4g128(const uint16_t* w, int64_t E, int64_t N, int64_t K,
+                                 uint32_t* packed, uint16_t* scales, moe_stream_t stream);
+
+/* 8-bitplane variable-precision form [PagedMoE bitplane prefixes; MatMoE floor and
+ * compensation].  Per group of 128: scale = bf16(max|w| / 127); q = clamp(rint(w /
+ * scale), -127, 127); u = q + 128 in 1..255.  Plane p (0..7) holds bit 7-p of u
+ * (plane 0 = most significant), element k of a row in bit k%32 of word k/32.
+ * A b-plane prefix is reconstructed as u' = ((u >> (8-b)) << (8-b)) + (b < 8 ? 1 << (7-b) : 0),
+ * w' = scale * (u' - 128).
+ *   w bf16 [E][N][K];  planes uint32 [E][8][N][K/32];  scales bf16 [E][N][K/128].
+ * Requires K % 128 == 0.  Bit-exact. */
+moe_status_t moe_pack_bitplanes(const uint16_t* w, int64_t E, int64_t N, int64_t K,
+                                uint32_t* planes, uint16_t* scales, moe_stream_t stream);
+
+/* NVFP4 quantisation [MoET, NVFP4 reference].  Per expert matrix (one [N][K] slice):
+ * g = amax / (6 * 448) (fp32).  Per block of 16 consecutive K elements:
+ * sb = E4M3_satfinite(amax_block / (6 * g)); code = E2M1_satfinite(w / (float(sb) * g)),
+ * round to nearest even, a magnitude that rounds to zero is +0 (code 0); g == 0 or
+ * sb == 0 gives codes 0.  Element 2i sits in the low nibble of byte i.
+ *   w bf16 [E][N][K];  codes uint8 [E][N][K/2];  block_scales uint8 [E][N][K/16];  gscale fp32 [E].
+ * gscale is also used as scratch during the call.  Requires K % 32 == 0.  Bit-exact. */
+moe_status_t moe_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64_t K,
+                                uint8_t* codes, uint8_t* block_scales, float* gscale,
+                                moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * One layer step: route -> (select_bits) -> grouped_ffn -> combine
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of device workspace moe_route_topk needs for (T, E, k). */
+size_t moe_route_workspace_bytes(int64_t T, int64_t E, int64_t k);
+
+/* Router logits, top-k, softmax weights and the stable permutation [ExactMoE: BF16
+ * router, unchanged top-k; nothing pruned or substituted].
+ * logits[t][e] = sum_h x[t][h] * w_router[e][h] (+ bias[e]) in fp32, in one fixed
+ * order: 32 partial sums, partial L accumulating h = 256j + 8L + i for j outer,
+ * i = 0..7 inner, by fused multiply-add from +0; the partials then added pairwise
+ * at lane distance 16, 8, 4, 2, 1; then + bias.  Top-k: logit descending, equal
+ * logits by ascending expert id.  Weights: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ * over the k chosen.  Permutation: stable counting sort of the pairs by expert.
+ *   x bf16 [T][H];  w_router bf16 [E][H];  bias fp32 [E] or NULL;  out: see moe_routing_t.
+ * Requires H % 256 == 0, 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= min(E, MOE_MAX_TOPK),
+ * T >= 0; workspace >= moe_route_workspace_bytes(T, E, k) (contents need not be
+ * initialised; overwritten).  Ids and permutation are deterministic. */
+moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                            int64_t T, int64_t H, int64_t E, int64_t k,
+                            const moe_routing_t* out, void* workspace, size_t workspace_bytes,
+                            moe_stream_t stream);
+
+/* Per-pair bit-width from the routing weight [MatMoE: precision per expert from
+ * routing scores; PagedMoE: prefix length from current routing weights].
+ * bits[p] = choices[0] if w < thresholds[0], choices[1] if w < thresholds[1],
+ * choices[2] if w < thresholds[2], else choices[3] (fp32 compares; equality takes
+ * the higher tier).  thresholds and choices are HOST arrays (copied at the call);
+ * thresholds ascending, choices in 1..8.
+ *   topk_w fp32 [T*k];  bits uint8 [T*k]. */
+moe_status_t moe_select_bits(const float* topk_w, int64_t T, int64_t k,
+                             const float thresholds[3], const uint8_t choices[4],
+                             uint8_t* bits, moe_stream_t stream);
+
+/* Bytes of device workspace moe_grouped_ffn needs. */
+size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                               moe_format_t fmt);
+
+/* Grouped SwiGLU expert FFN over the permuted pairs [ExactMoE: fused grouped
+ * execution of all selected experts; PagedMoE: prefixes executed directly, no
+ * full-precision expert materialised].
+ * For sorted row r of expert e holding pair p = t*k + j:
+ *   g = x[t] . deq(W_gate_e)^T, u = x[t] . deq(W_up_e)^T  (fp32 accumulation),
+ *   h = bf16(silu(g) * u),  y_rows[r] = bf16(h . deq(W2_e)^T).
+ * Dequantisation happens in registers; for BITPLANE8 expert e is read at bits[p]
+ * planes for pair p (planes 0..bits[p]-1, floor and compensation as above).
+ *   x bf16 [T][H];  routing: as written by moe_route_topk;  bits uint8 [T*k]
+ *   (BITPLANE8 only, values 1..8, else may be NULL);  y_rows bf16 [T*k][H].
+ * Requires H % 256 == 0, I % 128 == 0, the limits of moe_route_topk, and workspace
+ * >= moe_ffn_workspace_bytes(...).  Not bit-exact: fp32 accumulation order and the
+ * bf16 rounding of h differ from an fp64 reference (ExactMoE: the low-bit layer is
+ * not numerically identical to BF16). */
+moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
+                             const moe_experts_t* experts, const uint8_t* bits,
+                             int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                             uint16_t* y_rows, void* workspace, size_t workspace_bytes,
+                             moe_stream_t stream);
+
+/* Routing-weighted combine [ExactMoE: the selected experts' outputs weighted by the
+ * unchanged routing weights]: out[t] = bf16( sum_{j<k} topk_w[t*k+j] *
+ * y_rows[pair_to_row[t*k+j]] (+ residual[t]) ), fp32 accumulation in slot order j.
+ *   y_rows bf16 [T*k][H];  residual bf16 [T][H] or NULL;  out bf16 [T][H] (may alias residual).
+ * Requires H % 8 == 0.  Deterministic. */
+moe_status_t moe_combine(const uint16_t* y_rows, const moe_routing_t* routing,
+                         const uint16_t* residual, int64_t T, int64_t H, int64_t k,
+                         uint16_t* out, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Device error reporting
+ * ------------------------------------------------------------------------ */
+
+/* Synchronises `stream`, then reads and clears the library's device error word.
+ * Kernels never trap: a kernel whose bounded wait on an asynchronous copy runs out
+ * records the fact and returns.  Returns MOE_ERR_DEVICE_TIMEOUT if any kernel on
+ * this device recorded one since the last call, MOE_ERR_CUDA if the stream reports
+ * an error, else MOE_OK. */
+moe_status_t moe_check_device_errors(moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

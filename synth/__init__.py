@@ -62,16 +62,22 @@ def uniform01(seed: int, idx: np.ndarray) -> np.ndarray:
     return (w >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
 
 
+def _ih12_chunk(seed: int, idx: np.ndarray) -> np.ndarray:
+    """Sum of the twelve 16-bit fields of words 3i, 3i+1, 3i+2 (two fields per
+    32-bit half added first, then the halves), as int64."""
+    lanes = np.uint64(0x0000FFFF0000FFFF)
+    acc = np.zeros(idx.shape, dtype=np.uint64)
+    base = idx * np.uint64(3)
+    for m in range(3):
+        w = words(seed, base + np.uint64(m))
+        acc += (w & lanes) + ((w >> np.uint64(16)) & lanes)
+    return ((acc & np.uint64(0xFFFFFFFF)) + (acc >> np.uint64(32))).astype(np.int64)
+
+
 def irwin_hall12(seed: int, idx: np.ndarray) -> np.ndarray:
     """Exact float64 deviate with mean 0 and variance 1 for indices ``idx``."""
     idx = np.asarray(idx, dtype=np.uint64)
-    total = np.zeros(idx.shape, dtype=np.int64)
-    mask = np.uint64(0xFFFF)
-    for m in range(3):
-        w = words(seed, idx * np.uint64(3) + np.uint64(m))
-        for q in range(4):
-            total += ((w >> np.uint64(16 * q)) & mask).astype(np.int64)
-    return (total - 393210).astype(np.float64) / 65536.0
+    return (_ih12_chunk(seed, idx) - 393210).astype(np.float64) / 65536.0
 
 
 def f32_to_bf16_bits(f: np.ndarray) -> np.ndarray:
@@ -89,17 +95,43 @@ def _index(start: int, n: int) -> np.ndarray:
     return np.arange(start, start + n, dtype=np.uint64)
 
 
+_CHUNK = 1 << 20
+
+
+def _parallel_chunks(n: int, fn) -> np.ndarray:
+    """Evaluates fn(lo, hi) -> uint16 array over [0, n) in chunks on a thread pool
+    (numpy releases the GIL inside its loops); the result does not depend on the
+    chunking."""
+    out = np.empty(n, dtype=np.uint16)
+    spans = [(lo, min(n, lo + _CHUNK)) for lo in range(0, n, _CHUNK)]
+    if len(spans) <= 1:
+        for lo, hi in spans:
+            out[lo:hi] = fn(lo, hi)
+        return out
+    import concurrent.futures as cf
+    import os
+    with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        for (lo, hi), part in zip(spans, ex.map(lambda s: fn(*s), spans)):
+            out[lo:hi] = part
+    return out
+
+
 def normal_bf16(seed: int, n: int, std: float, start: int = 0) -> np.ndarray:
     """``n`` bf16 bit patterns (uint16) of std * Irwin-Hall(12) deviates, elements start..start+n-1."""
-    z = irwin_hall12(seed, _index(start, n))
-    return f32_to_bf16_bits((z * np.float64(std)).astype(np.float32))
+    def part(lo, hi):
+        z = irwin_hall12(seed, _index(start + lo, hi - lo))
+        return f32_to_bf16_bits((z * np.float64(std)).astype(np.float32))
+    return _parallel_chunks(n, part)
 
 
 def uniform_bf16(seed: int, n: int, lo: float, hi: float, start: int = 0) -> np.ndarray:
     """``n`` bf16 bit patterns of lo + (hi - lo) * U[0,1), elements start..start+n-1."""
-    u = uniform01(seed, _index(start, n))
     d = np.float64(hi) - np.float64(lo)
-    return f32_to_bf16_bits((np.float64(lo) + d * u).astype(np.float32))
+
+    def part(a, b):
+        u = uniform01(seed, _index(start + a, b - a))
+        return f32_to_bf16_bits((np.float64(lo) + d * u).astype(np.float32))
+    return _parallel_chunks(n, part)
 
 
 def normal_rows_bf16(seed: int, shape_tail: tuple, std: float, first_row: int, n_rows: int) -> np.ndarray:

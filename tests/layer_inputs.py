@@ -1,0 +1,85 @@
+"""Seeded inputs of one MoE layer, made once on the host (numpy, module `synth`)
+and handed to both sides: the oracle gets the numpy arrays, the CUDA path gets
+device copies of the same bytes.  Also the tolerance check shared by the tests."""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+import synth
+from oracle.ffn import FMT_BITPLANE8, FMT_NVFP4, FMT_W4G128, Experts
+from oracle.quant import pack_bitplanes, quantize_nvfp4, quantize_w4g128
+
+# Output tolerance of the FFN / combine against the float64 oracle.
+ATOL = 2e-2
+REL_L2 = 1e-2
+
+
+def dev_bf16(a: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def as_u32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().numpy().view(np.uint32)
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+@dataclass
+class LayerInputs:
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    x: np.ndarray        # bf16 bits [T][H]
+    wr: np.ndarray       # bf16 bits [E][H]
+    bias: np.ndarray | None
+    w13: np.ndarray      # bf16 bits [E][2I][H]
+    w2: np.ndarray       # bf16 bits [E][H][I]
+
+
+def make_layer(seed: int, T: int, H: int, I: int, E: int, k: int, router: str = "normal",
+               zipf: bool = False, wstd: float = 0.02, with_experts: bool = True) -> LayerInputs:
+    x = synth.normal_bf16(seed + synth.SEED_X, T * H, 1.0).reshape(T, H)
+    if router == "uniform":
+        wr = synth.uniform_bf16(seed + synth.SEED_WR, E * H, -0.02, 0.02).reshape(E, H)
+    else:
+        wr = synth.normal_bf16(seed + synth.SEED_WR, E * H, 0.02).reshape(E, H)
+    bias = synth.zipf_rank_bias(seed + synth.SEED_BIAS, E) if zipf else None
+    w13 = w2 = None
+    if with_experts:
+        w13 = synth.normal_bf16(seed + synth.SEED_W13, E * 2 * I * H, wstd).reshape(E, 2 * I, H)
+        w2 = synth.normal_bf16(seed + synth.SEED_W2, E * H * I, wstd).reshape(E, H, I)
+    return LayerInputs(T, H, I, E, k, x, wr, bias, w13, w2)
+
+
+def oracle_experts(fmt: int, w13: np.ndarray, w2: np.ndarray) -> Experts:
+    if fmt == FMT_W4G128:
+        a, b = quantize_w4g128(w13), quantize_w4g128(w2)
+        return Experts(fmt, a[0], a[1], b[0], b[1])
+    if fmt == FMT_BITPLANE8:
+        a, b = pack_bitplanes(w13), pack_bitplanes(w2)
+        return Experts(fmt, a[0], a[1], b[0], b[1])
+    a, b = quantize_nvfp4(w13), quantize_nvfp4(w2)
+    return Experts(fmt, a[0], a[1], b[0], b[1], a[2], b[2])
+
+
+def check_close(got: np.ndarray, ref: np.ndarray, what: str, atol=ATOL, rel_l2=REL_L2):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= atol, f"{what}: max abs err {err.max():.3e} > {atol}"
+    assert rel <= rel_l2, f"{what}: rel L2 err {rel:.3e} > {rel_l2}"
+    return float(err.max()), float(rel)

@@ -1,0 +1,115 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every function
+that include/*.h declares, and rejects invalid arguments on the host before any
+CUDA call (argument validation never touches the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_mixed_precision_router_b200 as moe
+from bit_mixed_precision_router_b200 import ExpertsT, RoutingT
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, SHAPE, WS, CUDA, MISALIGNED = 0, 1, 2, 3, 4, 5
+A = 0x10000  # a fake, 16-byte aligned device address: validation only inspects the number
+
+
+def declared_functions():
+    names = set()
+    for h in ("moe.h", "moe_synth.h"):
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_mixed_precision_router_b200 import build
+    build.build()
+    return moe.load()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+    assert set(moe.exported_symbols()) == names  # the binding covers the whole ABI
+    assert lib.moe_abi_version() == 1
+    assert lib.moe_status_string(3) == b"workspace missing or too small"
+    assert lib.moe_status_string(99) == b"unknown status"
+
+
+def test_quantizer_validation(lib):
+    assert lib.moe_quantize_w4g128(A, 2, 4, 100, A, A, None) == SHAPE
+    assert lib.moe_quantize_w4g128(None, 2, 4, 128, A, A, None) == INVALID
+    assert lib.moe_quantize_w4g128(A, 0, 4, 128, A, A, None) == INVALID
+    assert lib.moe_quantize_w4g128(A + 2, 2, 4, 128, A, A, None) == MISALIGNED
+    assert lib.moe_pack_bitplanes(A, 2, 4, 96, A, A, None) == SHAPE
+    assert lib.moe_quantize_nvfp4(A, 2, 4, 48, A, A, A, None) == SHAPE
+    assert lib.moe_quantize_nvfp4(A, 2, 4, 64, A, A, None, None) == INVALID
+
+
+def _routing():
+    return RoutingT(A, A, A, A, A, A)
+
+
+def test_route_validation(lib):
+    r = _routing()
+    call = lambda T, H, E, k, ws=A, wsb=1 << 30, x=A: lib.moe_route_topk(x, A, None, T, H, E, k, ctypes.byref(r),
+                                                                         ws, wsb, None)
+    assert call(4, 200, 8, 2) == SHAPE        # H % 256
+    assert call(4, 256, 0, 1) == SHAPE        # E < 1
+    assert call(4, 256, 1025, 2) == SHAPE     # E > MOE_MAX_EXPERTS
+    assert call(4, 256, 8, 9) == SHAPE        # k > E
+    assert call(4, 256, 64, 33) == SHAPE      # k > MOE_MAX_TOPK
+    assert call(-1, 256, 8, 2) == INVALID
+    assert call(4, 256, 8, 2, ws=None) == WS
+    assert call(4, 256, 8, 2, wsb=16) == WS
+    assert call(4, 256, 8, 2, x=None) == INVALID
+    assert call(0, 256, 8, 2, ws=None, wsb=0) == OK  # no tokens: nothing to do, nothing launched
+    r.sorted_pair = None
+    assert call(4, 256, 8, 2) == INVALID
+    r.sorted_pair = A + 4
+    assert call(4, 256, 8, 2) == MISALIGNED
+    assert lib.moe_route_workspace_bytes(16, 64, 8) >= 16 * 64 * 4
+
+
+def test_ffn_and_combine_validation(lib):
+    r = _routing()
+    ex = ExpertsT(0, A, A, A, A, None, None)
+    call = lambda T, H, I, E, k, bits=None, ws=A, wsb=1 << 40: lib.moe_grouped_ffn(
+        A, ctypes.byref(r), ctypes.byref(ex), bits, T, H, I, E, k, A, ws, wsb, None)
+    assert call(4, 2048, 1000, 64, 8) == SHAPE   # I % 128
+    assert call(4, 2000, 1024, 64, 8) == SHAPE   # H % 256
+    assert call(4, 2048, 1024, 64, 8, ws=None) == WS
+    assert call(4, 2048, 1024, 64, 8, wsb=1024) == WS
+    assert call(0, 2048, 1024, 64, 8, ws=None, wsb=0) == OK
+    assert call(4, 65536, 1024, 64, 8) == SHAPE  # weight tile would not fit in shared memory
+    ex.fmt = 1
+    assert call(4, 2048, 1024, 64, 8) == INVALID  # bitplanes need the bits array
+    ex.fmt = 2
+    assert call(4, 2048, 1024, 64, 8) == INVALID  # NVFP4 needs the per-expert scales
+    ex.fmt = 7
+    assert call(4, 2048, 1024, 64, 8) == INVALID
+    assert lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 0) >= 16 * 8 * 1024 * 2
+    assert lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 2) > lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 0)
+    c = lambda T, H, k, res=None: lib.moe_combine(A, ctypes.byref(r), res, T, H, k, A, None)
+    assert c(4, 2044, 8) == SHAPE
+    assert c(4, 2048, 0) == INVALID
+    assert c(4, 2048, 8, res=A + 8) == MISALIGNED
+    assert c(0, 2048, 8) == OK
+
+
+def test_select_bits_validation(lib):
+    thr = (ctypes.c_float * 3)(0.05, 0.15, 0.3)
+    bad_thr = (ctypes.c_float * 3)(0.3, 0.15, 0.05)
+    ch = (ctypes.c_uint8 * 4)(2, 3, 4, 8)
+    bad_ch = (ctypes.c_uint8 * 4)(0, 3, 4, 8)
+    assert lib.moe_select_bits(A, 4, 8, bad_thr, ch, A, None) == INVALID
+    assert lib.moe_select_bits(A, 4, 8, thr, bad_ch, A, None) == INVALID
+    assert lib.moe_select_bits(A, 0, 8, thr, ch, A, None) == OK
+    assert lib.moe_synth_normal_bf16(None, 4, 0, 1, 1.0, None) == INVALID
+    assert lib.moe_synth_normal_bf16(A, 0, 0, 1, 1.0, None) == OK
