@@ -55,6 +55,8 @@ _SIGS = {
     "moe_route_workspace_bytes": ([_i64, _i64, _i64], _sz),
     "moe_route_topk": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.POINTER(RoutingT), _vp, _sz, _vp],
                        ctypes.c_int),
+    "moe_route_topk_noalloc": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.POINTER(RoutingT), _vp],
+                               ctypes.c_int),
     "moe_select_bits": ([_vp, _i64, _i64, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_uint8), _vp,
                          _vp], ctypes.c_int),
     "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
@@ -188,6 +190,20 @@ def moe_route_topk(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor |
     rc = out.c()
     _call("moe_route_topk", _p(_bits(x)), _p(_bits(w_router)), _p(bias), T, H, E, k, ctypes.byref(rc),
           _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return out
+
+
+def moe_route_topk_noalloc(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None, k: int,
+                           out: Routing | None = None, stream=None) -> Routing:
+    """moe_route_topk for callers that cannot provide device workspace: the logits
+    scratch is the library's fixed device array (T * E <= 65536); nothing is allocated
+    by the library.  Calls that overlap on one GPU race on that array."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    out = Routing.empty(T, E, k, x.device) if out is None else out
+    rc = out.c()
+    _call("moe_route_topk_noalloc", _p(_bits(x)), _p(_bits(w_router)), _p(bias), T, H, E, k, ctypes.byref(rc),
+          _stream(stream))
     return out
 
 

@@ -165,6 +165,28 @@ moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const f
                             const moe_routing_t* out, void* workspace, size_t workspace_bytes,
                             moe_stream_t stream);
 
+/* Maximum T * E accepted by moe_route_topk_noalloc (floats in its fixed array). */
+#define MOE_NOALLOC_MAX_LOGITS 65536
+
+/* moe_route_topk without a workspace argument.  No counterpart on the source pages:
+ * it exists for callers that cannot allocate device memory -- an engine that plans
+ * all device memory up front and hands a layer only fixed buffers, a custom-op host
+ * that passes just inputs and outputs, or code running while a stream is captured
+ * into a CUDA graph in global mode, where cudaMalloc is not allowed.
+ * Same computation, arguments, results and errors as moe_route_topk, except that
+ * the fp32 logits scratch is a fixed device array inside the library (256 KiB per
+ * GPU that loads the library, held until exit):
+ *   - T * E must be <= MOE_NOALLOC_MAX_LOGITS, else MOE_ERR_UNSUPPORTED_SHAPE;
+ *   - the library allocates nothing and frees nothing during the call;
+ *   - all calls share the array: calls whose kernels overlap on one GPU (e.g. on two
+ *     streams) race on it; serialise them;
+ *   - the first call on a device looks up the array's address (cudaGetSymbolAddress
+ *     with that device current) and caches it; make that first call before any
+ *     stream capture. */
+moe_status_t moe_route_topk_noalloc(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                                    int64_t T, int64_t H, int64_t E, int64_t k,
+                                    const moe_routing_t* out, moe_stream_t stream);
+
 /* Per-pair bit-width from the routing weight [MatMoE: precision per expert from
  * routing scores; PagedMoE: prefix length from current routing weights].
  * bits[p] = choices[0] if w < thresholds[0], choices[1] if w < thresholds[1],
