@@ -31,8 +31,6 @@ unsigned* device_error_word() {
 
 namespace {
 
-constexpr size_t kMaxDynSmem = 220 * 1024;
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -65,12 +63,6 @@ moe_status_t check_route_shape(int64_t T, int64_t E, int64_t k) {
   if (k < 1 || k > E || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T > INT_MAX / k) return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
-}
-
-size_t ffn_smem_need(int64_t K, moe_format_t fmt) {
-  // padded rows as laid out by the FFN kernels (16 rows; 8 planes for bitplanes)
-  if (fmt == MOE_FMT_BITPLANE8) return size_t(8 * 16) * size_t(K / 8 + 16);
-  return size_t(16) * size_t(K / 2 + 64);
 }
 
 }  // namespace
@@ -166,8 +158,7 @@ moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing, co
   if (!ex.w13 || !ex.w13_scale || !ex.w2 || !ex.w2_scale) return MOE_ERR_INVALID_ARG;
   if (ex.fmt == MOE_FMT_NVFP4 && (!ex.w13_gscale || !ex.w2_gscale)) return MOE_ERR_INVALID_ARG;
   if (H < 256 || H % 256 != 0 || I < 128 || I % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (ffn_smem_need(H, ex.fmt) > kMaxDynSmem || ffn_smem_need(I, ex.fmt) > kMaxDynSmem)
-    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (H > 65536 || I > 65536 || !moe::ffn_shape_supported(H, I, ex.fmt)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (int64_t(E) * 2 * I > INT_MAX || T * k > INT_MAX / (H > I ? H : I)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return MOE_OK;  // no pairs; no activation or output pointer is read
   if (!x || !y_rows) return MOE_ERR_INVALID_ARG;

@@ -1,16 +1,18 @@
 // Grouped expert FFN, weight-streaming path (decode-sized expert groups).
 //
-// One CTA = one routed expert x one tile of 16 weight rows, full K:
-//   gate/up: smem rows 0..7 = gate rows 8t..8t+7, rows 8..15 = the matching up rows,
-//            so one m16 MMA fragment yields gate and up of 8 intermediate rows and
-//            SwiGLU is applied in the epilogue;
-//   down:    smem rows 0..15 = down rows 16t..16t+15.
-// Warp 0 issues one bulk copy (TMA engine) per weight row (per plane for the
-// bitplane format) into padded shared memory, so the whole tile is in flight at
-// once; the 4 warps split K, dequantise in registers and feed mma.sync with the
-// expert's tokens on the MMA's N dimension (16 per pass); partial sums meet in
-// shared memory in a fixed warp order.  Expert weights are read once per CTA no
-// matter how many tokens the expert received.
+// Work: every routed expert's weight matrix is cut into units of 16 rows x full K
+//   gate/up: rows 0..7 = gate rows 8t..8t+7, rows 8..15 = the matching up rows (one m16
+//            MMA fragment gives gate and up of 8 intermediate rows, so SwiGLU runs in
+//            the epilogue);
+//   down:    rows 0..15 = down rows 16t..16t+15.
+// One CTA = one routed expert x 8 warps, each warp owning whole units.  The expert's
+// activations for a chunk of up to `nx` tokens are staged once per CTA in shared memory,
+// already paired the way the dequantised weights pair them and with their per-group sums.
+// Each warp then streams its own units group by group (16 rows x 128 K-elements per step)
+// through a private ring of shared-memory slots with 16-byte cp.async copies kept kDepth
+// steps ahead (commit/wait groups, no cross-warp handshake), and per step: shared loads,
+// nibble / bit / FP4 -> bf16 (fp16) in registers, mma.sync m16n8k16 with the tokens on N.
+// Expert weights are read from HBM once per token chunk.
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
@@ -20,12 +22,15 @@
 namespace moe {
 
 enum { kGateUp = 0, kDown = 1 };
-constexpr int kRows = 16;    // weight rows per CTA
-constexpr int kWarps = 4;    // K split
-constexpr int kChunk = 16;   // tokens per pass (two n8 tiles)
+constexpr int kRows = 16;     // weight rows per unit
+constexpr int kWarps = 8;     // warps per CTA, each owning whole units
+constexpr int kThreads = 32 * kWarps;
+constexpr int kDepth = 6;     // group steps in flight per warp
+constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
+constexpr size_t kSmemTarget = 110 * 1024;  // two CTAs per SM
 
 struct FfnArgs {
-  const void* act;  // gate/up: x [T][K] (bf16, or fp16*2^-8 for NVFP4); down: h [P][K]
+  const void* act;  // gate/up: x bf16 [T][K]; down: h [P][K] (bf16, or fp16*2^-8 for NVFP4)
   int K;            // reduction length: H (gate/up) or I (down)
   int N;            // rows per expert matrix: 2I or H
   int I;
@@ -39,57 +44,49 @@ struct FfnArgs {
   const float* gscale;  // NVFP4
   void* out;            // gate/up: h [P][I]; down: y [P][H]
   int out_ld;
-  unsigned* err;
+  // shared-memory plan (bytes), filled by the launcher
+  int nx, x_stride, slot_bytes, warp_bytes, off_x, off_xsum, off_bits;
 };
 
-// Row stride (bytes) of a K-contiguous weight row of `row_bytes` in shared memory,
-// padded so that the 16-byte (W4/NVFP4) or 4-byte (bitplane) loads of the 32 lanes
-// hit distinct banks.
-__host__ __device__ inline int smem_stride_16B(int row_bytes) {
-  // row_bytes / 16 is a multiple of 4; make the stride / 16 an odd multiple of 4 (mod 8 == 4)
-  return ((row_bytes / 16) % 8 == 4) ? row_bytes : row_bytes + 64;
+template <int FMT>
+__host__ __device__ inline int slot_bytes_of() {  // one group step of one unit
+  return FMT == MOE_FMT_BITPLANE8 ? 8 * kRows * 16 : (FMT == MOE_FMT_NVFP4 ? kRows * 64 + kRows * 8 : kRows * 64);
 }
-__host__ __device__ inline int smem_stride_4B(int row_bytes) {
-  // stride / 4 must be 4 * odd (mod 32 in {4, 12, 20, 28})
-  return (((row_bytes / 16) & 1) == 1) ? row_bytes : row_bytes + 16;
+// x rows: stride/16 = 4 (mod 8) keeps the 8 lanes of a quarter warp on distinct banks
+__host__ __device__ inline int stride_16B(int row_bytes) {
+  return ((row_bytes / 16) % 8 == 4) ? row_bytes : row_bytes + ((4 - (row_bytes / 16) % 8) + 8) % 8 * 16;
 }
 
-template <int FMT>
-__host__ __device__ inline int weight_row_bytes(int K) {
-  return FMT == MOE_FMT_BITPLANE8 ? K / 8 : K / 2;
+// ---------------------------------------------------------------- async copies
+MOE_DEVICE void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
-template <int FMT>
-__host__ __device__ inline int weight_stride(int K) {
-  return FMT == MOE_FMT_BITPLANE8 ? smem_stride_4B(K / 8) : smem_stride_16B(K / 2);
+MOE_DEVICE void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
-template <int FMT>
-__host__ inline size_t ffn_smem_bytes(int K) {
-  const int planes = FMT == MOE_FMT_BITPLANE8 ? 8 : 1;
-  return size_t(planes) * kRows * weight_stride<FMT>(K);
-}
+MOE_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+MOE_DEVICE void cp_async_wait_depth() { asm volatile("cp.async.wait_group %0;" ::"n"(kDepth - 1) : "memory"); }
+MOE_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- group steps
-// Every step handles one group of 128 K-elements for the thread's 32-element slice
-// (lane = 4g + c owns K-elements 32c .. 32c+31 of the group) of smem rows g and
-// g+8, for up to two n8 tiles of tokens whose activation slices are in xv[nt][0..3].
+// One group of 128 K-elements for the thread's slice (lane = 4g + c owns elements
+// 32c .. 32c+31 of the group) of unit rows g and g+8, for one or two n8 token tiles.
+// xv[nt][m] holds the pre-paired activations of word m of the slice for token column g
+// of tile nt; X[nt][j] the group sum of the activations of token 2c+j of tile nt.
 
-// INT4: word m of the slice holds elements 8m .. 8m+7.  Nibbles j and j+4 are
-// lifted into one bf16x2 as 128 + u (exponent of 128, nibble in the low mantissa
-// bits); the MMA therefore sums (q + 136) * x and a second MMA with A = 136
-// removes the offset.  The activations are paired (j, j+4) to match.
-MOE_DEVICE void w4_group(const uint8_t* rowA, const uint8_t* rowB, const uint4 (&xv)[2][4], bool two, float sa,
-                         float sb, float (&acc)[2][4]) {
-  const uint4 wa = *reinterpret_cast<const uint4*>(rowA);
-  const uint4 wb = *reinterpret_cast<const uint4*>(rowB);
+// INT4: nibbles j and j+4 of a word become one bf16x2 of (128 + u) with one shift and one
+// LOP3; the activations were paired (j, j+4) when staged.  The MMA sums (q + 136) * x;
+// 136 * sum(x) is removed with the staged group sums.
+MOE_DEVICE void w4_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], bool two, float sa, float sb,
+                         const float (&X)[2][2], float (&acc)[2][4]) {
   const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
   const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
   constexpr uint32_t kMagic = 0x43004300u;  // bf16 (128, 128)
-  constexpr uint32_t kOff = 0x43084308u;    // bf16 (136, 136)
-  float tmp[2][4], corr[2][4];
+  float t0[2][4], t1[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) tmp[nt][i] = corr[nt][i] = 0.f;
+    for (int i = 0; i < 4; ++i) t0[nt][i] = t1[nt][i] = 0.f;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     uint32_t pa[4], pb[4];
@@ -102,74 +99,49 @@ MOE_DEVICE void w4_group(const uint8_t* rowA, const uint8_t* rowB, const uint4 (
     for (int nt = 0; nt < 2; ++nt) {
       if (nt == 1 && !two) break;
       const uint4 xx = xv[nt][m];
-      const uint32_t b00 = __byte_perm(xx.x, xx.z, 0x5410), b01 = __byte_perm(xx.x, xx.z, 0x7632);
-      const uint32_t b10 = __byte_perm(xx.y, xx.w, 0x5410), b11 = __byte_perm(xx.y, xx.w, 0x7632);
-      mma_bf16(tmp[nt], pa[0], pb[0], pa[1], pb[1], b00, b01);
-      mma_bf16(tmp[nt], pa[2], pb[2], pa[3], pb[3], b10, b11);
-      mma_bf16(corr[nt], kOff, kOff, kOff, kOff, b00, b01);
-      mma_bf16(corr[nt], kOff, kOff, kOff, kOff, b10, b11);
+      float(&t)[4] = (m & 1) ? t1[nt] : t0[nt];
+      mma_bf16(t, pa[0], pb[0], pa[1], pb[1], xx.x, xx.y);
+      mma_bf16(t, pa[2], pb[2], pa[3], pb[3], xx.z, xx.w);
     }
   }
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    acc[nt][0] = fmaf(sa, tmp[nt][0] - corr[nt][0], acc[nt][0]);
-    acc[nt][1] = fmaf(sa, tmp[nt][1] - corr[nt][1], acc[nt][1]);
-    acc[nt][2] = fmaf(sb, tmp[nt][2] - corr[nt][2], acc[nt][2]);
-    acc[nt][3] = fmaf(sb, tmp[nt][3] - corr[nt][3], acc[nt][3]);
+    const float c0 = 136.f * X[nt][0], c1 = 136.f * X[nt][1];
+    acc[nt][0] = fmaf(sa, (t0[nt][0] + t1[nt][0]) - c0, acc[nt][0]);
+    acc[nt][1] = fmaf(sa, (t0[nt][1] + t1[nt][1]) - c1, acc[nt][1]);
+    acc[nt][2] = fmaf(sb, (t0[nt][2] + t1[nt][2]) - c0, acc[nt][2]);
+    acc[nt][3] = fmaf(sb, (t0[nt][3] + t1[nt][3]) - c1, acc[nt][3]);
   }
 }
 
-// Bitplanes: plane word bit j <-> element j of the 32-element slice.  Bits j and
-// j+16 are moved to bit 7 / 23 of a bf16x2 whose other bits spell 0.5, giving
-// A = 0.5 + 0.5 * bit; activations are paired (j, j+16).  For token t read at
-// b_t planes the group contributes
-//   sum_{p < b_t} 2^(8-p) * T_p + (c_b + 2^(8-b) - 384) * X,
-// with T_p the plane-p MMA sum and X = sum of the activations over the slice
-// (an MMA with A = 1), which equals sum_k (u'_k - 128) x_k.
+// Bitplanes: plane-word bit j <-> element j of the slice.  Bits j and j+16 move to
+// bit 7 / 23 of a bf16x2 whose other bits spell 0.5, so A = 0.5 + 0.5 * bit; the
+// activations were paired (j, j+16) when staged.  With T_p the plane-p MMA sum and X
+// the group sum of the activations, a token read at b planes gets
+//   sum_{p < b} 2^(8-p) T_p + (c_b + 2^(8-b) - 384) X  =  sum_k (u'_k - 128) x_k,
+// c_b = 2^(7-b) for b < 8, 0 for b = 8 (floor plus half-step compensation).
 MOE_DEVICE uint32_t bit_pair(uint32_t w, int j) {
   const uint32_t s = (j <= 7) ? (w << (7 - j)) : (w >> (j - 7));
   return (s & 0x00800080u) | 0x3F003F00u;
 }
-MOE_DEVICE float plane_coef_x(int b) {  // c_b + 2^(8-b) - 384
-  return (b >= 8) ? -383.f : float(3 * (1 << (7 - b)) - 384);
-}
+MOE_DEVICE float plane_coef_x(int b) { return (b >= 8) ? -383.f : float(3 * (1 << (7 - b)) - 384); }
 
-MOE_DEVICE void bp_group(const uint8_t* base, int stride, int G, int g, int c, int nplanes,
-                         const uint4 (&xv)[2][4], bool two, const int (&bt)[2][2], float sa, float sb,
-                         float (&acc)[2][4]) {
-  uint32_t R[2][16];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const uint32_t* q = reinterpret_cast<const uint32_t*>(&xv[nt][0]);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) R[nt][i] = q[i];
-  }
-  constexpr uint32_t kOne = 0x3F803F80u;
-  float X[2][4], grp[2][4];
+// pl: the thread's word of plane 0, row g; planes are 16 rows x 16 bytes apart.
+MOE_DEVICE void bp_group(const uint8_t* pl, int nplanes, const uint4 (&xv)[2][4], bool two, const int (&bt)[2][2],
+                         float sa, float sb, const float (&X)[2][2], float (&acc)[2][4]) {
+  float grp[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) X[nt][i] = grp[nt][i] = 0.f;
-  // X = sum of activations (plane independent)
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      if (nt == 1 && !two) break;
-      const uint32_t b0 = __byte_perm(R[nt][s], R[nt][s + 8], 0x5410);
-      const uint32_t b1 = __byte_perm(R[nt][s], R[nt][s + 8], 0x7632);
-      mma_bf16(X[nt], kOne, kOne, kOne, kOne, b0, b1);
-    }
-  }
+    for (int i = 0; i < 4; ++i) grp[nt][i] = 0.f;
   for (int p = 0; p < nplanes; ++p) {
-    const uint8_t* pr = base + (p * kRows + g) * stride + G * 16 + c * 4;
-    const uint32_t wa = *reinterpret_cast<const uint32_t*>(pr);
-    const uint32_t wb = *reinterpret_cast<const uint32_t*>(pr + 8 * stride);
-    float tp[2][4];
+    const uint32_t wa = *reinterpret_cast<const uint32_t*>(pl + p * kRows * 16);
+    const uint32_t wb = *reinterpret_cast<const uint32_t*>(pl + p * kRows * 16 + 8 * 16);
+    float t0[2][4], t1[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tp[nt][i] = 0.f;
+      for (int i = 0; i < 4; ++i) t0[nt][i] = t1[nt][i] = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       const uint32_t a0 = bit_pair(wa, 2 * s), a2 = bit_pair(wa, 2 * s + 1);
@@ -177,34 +149,35 @@ MOE_DEVICE void bp_group(const uint8_t* base, int stride, int G, int g, int c, i
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         if (nt == 1 && !two) break;
-        const uint32_t b0 = __byte_perm(R[nt][s], R[nt][s + 8], 0x5410);
-        const uint32_t b1 = __byte_perm(R[nt][s], R[nt][s + 8], 0x7632);
-        mma_bf16(tp[nt], a0, a1, a2, a3, b0, b1);
+        const uint4 xx = xv[nt][s >> 1];
+        const uint32_t b0 = (s & 1) ? xx.z : xx.x, b1 = (s & 1) ? xx.w : xx.y;
+        float(&t)[4] = (s & 1) ? t1[nt] : t0[nt];
+        mma_bf16(t, a0, a1, a2, a3, b0, b1);
       }
     }
     const float f = float(1 << (8 - p));
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const float f0 = (p < bt[nt][0]) ? f : 0.f, f1 = (p < bt[nt][1]) ? f : 0.f;
-      grp[nt][0] = fmaf(f0, tp[nt][0], grp[nt][0]);
-      grp[nt][1] = fmaf(f1, tp[nt][1], grp[nt][1]);
-      grp[nt][2] = fmaf(f0, tp[nt][2], grp[nt][2]);
-      grp[nt][3] = fmaf(f1, tp[nt][3], grp[nt][3]);
+      grp[nt][0] = fmaf(f0, t0[nt][0] + t1[nt][0], grp[nt][0]);
+      grp[nt][1] = fmaf(f1, t0[nt][1] + t1[nt][1], grp[nt][1]);
+      grp[nt][2] = fmaf(f0, t0[nt][2] + t1[nt][2], grp[nt][2]);
+      grp[nt][3] = fmaf(f1, t0[nt][3] + t1[nt][3], grp[nt][3]);
     }
   }
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    const float x0 = plane_coef_x(bt[nt][0]), x1 = plane_coef_x(bt[nt][1]);
-    acc[nt][0] = fmaf(sa, fmaf(x0, X[nt][0], grp[nt][0]), acc[nt][0]);
-    acc[nt][1] = fmaf(sa, fmaf(x1, X[nt][1], grp[nt][1]), acc[nt][1]);
-    acc[nt][2] = fmaf(sb, fmaf(x0, X[nt][2], grp[nt][2]), acc[nt][2]);
-    acc[nt][3] = fmaf(sb, fmaf(x1, X[nt][3], grp[nt][3]), acc[nt][3]);
+    const float x0 = plane_coef_x(bt[nt][0]) * X[nt][0], x1 = plane_coef_x(bt[nt][1]) * X[nt][1];
+    acc[nt][0] = fmaf(sa, grp[nt][0] + x0, acc[nt][0]);
+    acc[nt][1] = fmaf(sa, grp[nt][1] + x1, acc[nt][1]);
+    acc[nt][2] = fmaf(sb, grp[nt][2] + x0, acc[nt][2]);
+    acc[nt][3] = fmaf(sb, grp[nt][3] + x1, acc[nt][3]);
   }
 }
 
-// NVFP4: byte i of a word holds elements 2i (low nibble) and 2i+1; each byte is
-// converted to an fp16 pair and multiplied by its E4M3 block scale (exact in fp16);
-// activations are fp16 (pre-scaled by 2^-8) in natural pairs.
+// NVFP4: byte i of a word holds elements 2i (low nibble) and 2i+1; the hardware converts
+// the pair to fp16 and the E4M3 block scale multiplies it in fp16 (exact); activations
+// are fp16 * 2^-8 in natural pairs.
 MOE_DEVICE uint32_t e2m1x2_to_h2(uint32_t byte) {
   const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
   return uint32_t(r.x) | (uint32_t(r.y) << 16);
@@ -219,13 +192,11 @@ MOE_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {
   return d;
 }
 
-MOE_DEVICE void fp4_group(const uint8_t* rowA, const uint8_t* rowB, uint32_t scA, uint32_t scB,
-                          const uint4 (&xv)[2][4], bool two, float (&acc)[2][4]) {
-  const uint4 wa = *reinterpret_cast<const uint4*>(rowA);
-  const uint4 wb = *reinterpret_cast<const uint4*>(rowB);
+MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const uint4 (&xv)[2][4], bool two,
+                          float (&acc)[2][4]) {
   const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
   const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
-  // block scales: words 0,1 -> block 2c (byte 0 of sc), words 2,3 -> block 2c+1 (byte 1)
+  // words 0,1 -> block 2c (byte 0 of sc), words 2,3 -> block 2c+1 (byte 1)
   const uint32_t sA[2] = {e4m3_to_h2(scA & 0xFF), e4m3_to_h2((scA >> 8) & 0xFF)};
   const uint32_t sB[2] = {e4m3_to_h2(scB & 0xFF), e4m3_to_h2((scB >> 8) & 0xFF)};
 #pragma unroll
@@ -248,11 +219,8 @@ MOE_DEVICE void fp4_group(const uint8_t* rowA, const uint8_t* rowB, uint32_t scA
 
 // ---------------------------------------------------------------- kernel
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(32 * kWarps) k_ffn_gemv(FfnArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint64_t bar;
-  __shared__ float red[kWarps][2][32][4];
-  __shared__ int s_bmax;
 
   const int slot = blockIdx.y;
   if (slot >= a.expert_list[0]) return;
@@ -260,197 +228,300 @@ __global__ void __launch_bounds__(32 * kWarps) k_ffn_gemv(FfnArgs a) {
   const int row0 = a.offsets[e];
   const int n_e = a.offsets[e + 1] - row0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int K = a.K;
-  const int stride = weight_stride<FMT>(K);
-  const int row_bytes = weight_row_bytes<FMT>(K);
+  const int K = a.K, GK = K / 128;
+  const int TPE = (MODE == kGateUp) ? a.I / 8 : a.N / kRows;
+  const int rt = blockIdx.x * kWarps + warp;  // this warp's unit
+  const bool has_unit = rt < TPE;
 
-  // expert-matrix row of smem row i
-  auto wrow = [&](int i) -> int {
-    if (MODE == kGateUp) return (i < 8) ? (8 * blockIdx.x + i) : (a.I + 8 * blockIdx.x + i - 8);
-    return kRows * blockIdx.x + i;
+  uint8_t* xbuf = smem + a.off_x;
+  float* xsum = reinterpret_cast<float*>(smem + a.off_xsum);
+  int* sbits = reinterpret_cast<int*>(smem + a.off_bits);
+  uint8_t* wsm = smem + size_t(warp) * a.warp_bytes;  // this warp's ring (+ scales)
+  uint16_t* wscale = reinterpret_cast<uint16_t*>(wsm + kDepth * a.slot_bytes);
+
+  auto wrow = [&](int i) -> int {  // expert-matrix row of unit row i
+    if (MODE == kGateUp) return (i < 8) ? (8 * rt + i) : (a.I + 8 * rt + i - 8);
+    return kRows * rt + i;
   };
 
-  int nplanes = 1;
-  if (FMT == MOE_FMT_BITPLANE8) {
-    int bm = 1;
-    for (int n = threadIdx.x; n < n_e; n += blockDim.x) bm = max(bm, int(a.bits[a.sorted_pair[row0 + n]]));
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) bm = max(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-    if (threadIdx.x == 0) s_bmax = 1;
-    __syncthreads();
-    if (lane == 0) atomicMax(&s_bmax, bm);
-    __syncthreads();
-    nplanes = min(8, s_bmax);
-  }
-
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (warp == 0) {
-    if (lane == 0) mbar_arrive_expect_tx(&bar, uint32_t(nplanes * kRows * row_bytes));
-    __syncwarp();
-    for (int q = lane; q < nplanes * kRows; q += 32) {
-      const int i = q % kRows, pl = q / kRows;
-      const uint8_t* src;
-      if (FMT == MOE_FMT_BITPLANE8)
-        src = static_cast<const uint8_t*>(a.w) + ((size_t(e) * 8 + pl) * a.N + wrow(i)) * size_t(row_bytes);
-      else
-        src = static_cast<const uint8_t*>(a.w) + (size_t(e) * a.N + wrow(i)) * size_t(row_bytes);
-      bulk_g2s(smem + (pl * kRows + i) * stride, src, uint32_t(row_bytes), &bar);
+  // ---- per-lane copy plan of this warp's unit
+  // W4 / NVFP4: per step the lane copies 16 bytes of rows r = lane/4 and r + 8 (chunk lane%4),
+  //             plus (NVFP4, lane < 16) the 8 block scales of row lane.
+  // Bitplanes:  per step the lane copies the 16-byte group word of row lane%16 for planes
+  //             lane/16, lane/16 + 2, ... below the chunk's prefix length.
+  const uint8_t* wbase = static_cast<const uint8_t*>(a.w);
+  const size_t rbK = size_t(FMT == MOE_FMT_BITPLANE8 ? K / 8 : K / 2);  // bytes per weight row (per plane)
+  const size_t pstride = size_t(a.N) * rbK;
+  const uint8_t* srcA = wbase;
+  const uint8_t* srcB = wbase;
+  const uint8_t* sbA = wbase;
+  if (has_unit) {
+    if (FMT == MOE_FMT_BITPLANE8) {
+      srcA = wbase + (size_t(e) * 8 + (lane >> 4)) * pstride + size_t(wrow(lane & 15)) * rbK;
+    } else {
+      const int r = lane >> 2;
+      srcA = wbase + (size_t(e) * a.N + wrow(r)) * rbK + (lane & 3) * 16;
+      srcB = wbase + (size_t(e) * a.N + wrow(r + 8)) * rbK + (lane & 3) * 16;
+      if (FMT == MOE_FMT_NVFP4)
+        sbA = static_cast<const uint8_t*>(a.s) + (size_t(e) * a.N + wrow(lane & 15)) * size_t(K / 16);
     }
   }
 
-  const int Gtot = K / 128;
-  const int gpw = (Gtot + kWarps - 1) / kWarps;
-  const int gb = min(Gtot, warp * gpw), ge = min(Gtot, gb + gpw);
-  const int rA = wrow(g), rB = wrow(g + 8);
+  for (int tok0 = 0; tok0 < n_e; tok0 += a.nx) {
+    const int nvalid = min(a.nx, n_e - tok0);
+    const bool two = nvalid > 8;
+    if (tok0 > 0) __syncthreads();  // the previous chunk's activations are no longer read
 
-  const bool ok = mbar_wait(&bar, 0, a.err);
-  if (!__syncthreads_and(ok)) return;
-
-  for (int n0 = 0; n0 < n_e; n0 += kChunk) {
-    const bool two = (n_e - n0) > 8;
-    // B operand rows: token column g of each n8 tile
-    const uint8_t* arow[2];
-    int bt[2][2] = {{8, 8}, {8, 8}};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int n = n0 + nt * 8 + g;
-      arow[nt] = nullptr;
-      if (n < n_e) {
-        const int r = row0 + n;
-        const int arow_idx = (MODE == kGateUp) ? a.sorted_pair[r] / a.k : r;
-        arow[nt] = static_cast<const uint8_t*>(a.act) + size_t(arow_idx) * K * 2;
-      }
+    // bitplanes: prefix length of this chunk (known before any weight is requested)
+    int nplanes = 1;
+    if (FMT == MOE_FMT_BITPLANE8) {
+      for (int n = 0; n < nvalid; ++n) nplanes = max(nplanes, int(a.bits[a.sorted_pair[row0 + tok0 + n]]));
+      nplanes = min(8, nplanes);
+    }
+    auto issue = [&](int G) {  // copy group G of the unit into ring slot G % kDepth
+      uint8_t* dst = wsm + (G % kDepth) * a.slot_bytes;
       if (FMT == MOE_FMT_BITPLANE8) {
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int nn = n0 + nt * 8 + 2 * c + jj;
-          bt[nt][jj] = (nn < n_e) ? int(a.bits[a.sorted_pair[row0 + nn]]) : 8;
+        const int i = lane & 15;
+        for (int p = lane >> 4; p < nplanes; p += 2)
+          cp_async16(dst + (p * kRows + i) * 16, srcA + size_t(p - (lane >> 4)) * pstride + G * 16);
+      } else {
+        const int r = lane >> 2;
+        cp_async16(dst + r * 64 + (lane & 3) * 16, srcA + G * 64);
+        cp_async16(dst + (r + 8) * 64 + (lane & 3) * 16, srcB + G * 64);
+        if (FMT == MOE_FMT_NVFP4 && lane < 16) cp_async8(dst + kRows * 64 + lane * 8, sbA + G * 8);
+      }
+    };
+    // start this warp's weight stream before staging activations (the two overlap)
+    if (has_unit) {
+      for (int G = 0; G < kDepth; ++G) {
+        if (G < GK) issue(G);
+        cp_async_commit();
+      }
+      if (FMT != MOE_FMT_NVFP4) {  // the unit's 16 rows x GK scales
+        const uint16_t* sb = static_cast<const uint16_t*>(a.s);
+        for (int idx = lane; idx < kRows * GK; idx += 32) {
+          const int i = idx / GK, gg = idx - i * GK;
+          wscale[idx] = sb[(size_t(e) * a.N + wrow(i)) * GK + gg];
         }
       }
     }
-    auto load_x = [&](uint4 (&xv)[2][4], int G) {
+
+    // ---- stage activations: slice q = (token n, 32-element slice sl), pre-paired per format
+    const int slices = K / 32;
+    const int nslices = nvalid * slices;
+    for (int q0 = 0; q0 < nslices; q0 += kThreads) {
+      const int q = q0 + threadIdx.x;
+      const bool ok = q < nslices;
+      float ssum = 0.f;
+      int n = 0, sl = 0;
+      if (ok) {
+        n = q / slices;
+        sl = q - n * slices;
+        const int r = row0 + tok0 + n;
+        const size_t arow = (MODE == kGateUp) ? size_t(a.sorted_pair[r] / a.k) : size_t(r);
+        const uint4* src =
+            reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.act) + (arow * K + size_t(sl) * 32) * 2);
+        uint32_t R[16];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int m = 0; m < 4; ++m) {
+          const uint4 v = src[m];
+          R[4 * m] = v.x;
+          R[4 * m + 1] = v.y;
+          R[4 * m + 2] = v.z;
+          R[4 * m + 3] = v.w;
+        }
+        uint32_t O[16];
+        if (FMT == MOE_FMT_W4G128) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {  // word m: (x0,x4), (x1,x5), (x2,x6), (x3,x7)
+            const uint32_t r0 = R[4 * m], r1 = R[4 * m + 1], r2 = R[4 * m + 2], r3 = R[4 * m + 3];
+            O[4 * m] = __byte_perm(r0, r2, 0x5410);
+            O[4 * m + 1] = __byte_perm(r0, r2, 0x7632);
+            O[4 * m + 2] = __byte_perm(r1, r3, 0x5410);
+            O[4 * m + 3] = __byte_perm(r1, r3, 0x7632);
+          }
+        } else if (FMT == MOE_FMT_BITPLANE8) {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {  // step s: (x_2s, x_2s+16), (x_2s+1, x_2s+17)
+            O[2 * s] = __byte_perm(R[s], R[s + 8], 0x5410);
+            O[2 * s + 1] = __byte_perm(R[s], R[s + 8], 0x7632);
+          }
+        } else {
+          if (MODE == kGateUp) {  // bf16 -> fp16 * 2^-8, natural pairs
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const __half2 h = __floats2half2_rn(bf16_lo(R[i]) * (1.0f / 256.f), bf16_hi(R[i]) * (1.0f / 256.f));
+              O[i] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) O[i] = R[i];
+          }
+        }
+        if (FMT != MOE_FMT_NVFP4) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ssum += bf16_lo(R[i]) + bf16_hi(R[i]);
+        }
+        // slice sl = group G, lane slice cc; word m of the slice goes to 16-byte chunk 4m + cc
+        const int G = sl >> 2, cc = sl & 3;
+        uint8_t* dst = xbuf + size_t(n) * a.x_stride + G * 256;
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          xv[nt][m] = arow[nt] ? *reinterpret_cast<const uint4*>(arow[nt] + (size_t(G) * 128 + c * 32 + m * 8) * 2)
-                               : make_uint4(0, 0, 0, 0);
-    };
+          *reinterpret_cast<uint4*>(dst + (4 * m + cc) * 16) =
+              make_uint4(O[4 * m], O[4 * m + 1], O[4 * m + 2], O[4 * m + 3]);
+      }
+      if (FMT != MOE_FMT_NVFP4) {  // group sums: the 4 slices of a group are 4 consecutive lanes
+        ssum += __shfl_xor_sync(0xffffffffu, ssum, 1);
+        ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
+        if (ok && (sl & 3) == 0) xsum[n * GK + (sl >> 2)] = ssum;
+      }
+    }
+    if (FMT == MOE_FMT_BITPLANE8)
+      for (int n = threadIdx.x; n < kMaxTok; n += kThreads)
+        sbits[n] = (n < nvalid) ? int(a.bits[a.sorted_pair[row0 + tok0 + n]]) : 8;
+    __syncthreads();
+    if (!has_unit) continue;
 
+    int bt[2][2] = {{8, 8}, {8, 8}};
+    if (FMT == MOE_FMT_BITPLANE8) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        bt[nt][0] = sbits[nt * 8 + 2 * c];
+        bt[nt][1] = sbits[nt * 8 + 2 * c + 1];
+      }
+    }
+
+    // ---- stream the unit: group G is computed while groups G+1 .. G+kDepth-1 are in flight
     float acc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-
-    uint4 xc[2][4], xn[2][4];
-    if (gb < ge) load_x(xc, gb);
-    for (int G = gb; G < ge; ++G) {
-      if (G + 1 < ge) load_x(xn, G + 1);
-      if (FMT == MOE_FMT_W4G128) {
-        const uint16_t* s = static_cast<const uint16_t*>(a.s);
-        const float sa = bf16_bits_to_float(s[(size_t(e) * a.N + rA) * Gtot + G]);
-        const float sb = bf16_bits_to_float(s[(size_t(e) * a.N + rB) * Gtot + G]);
-        const uint8_t* rowA = smem + g * stride + G * 64 + c * 16;
-        w4_group(rowA, rowA + 8 * stride, xc, two, sa, sb, acc);
-      } else if (FMT == MOE_FMT_BITPLANE8) {
-        const uint16_t* s = static_cast<const uint16_t*>(a.s);
-        const float sa = bf16_bits_to_float(s[(size_t(e) * a.N + rA) * Gtot + G]);
-        const float sb = bf16_bits_to_float(s[(size_t(e) * a.N + rB) * Gtot + G]);
-        bp_group(smem, stride, G, g, c, nplanes, xc, two, bt, sa, sb, acc);
-      } else {
-        const uint8_t* s = static_cast<const uint8_t*>(a.s);
-        const size_t spr = size_t(K / 16);
-        const uint32_t scA = *reinterpret_cast<const uint16_t*>(s + (size_t(e) * a.N + rA) * spr + G * 8 + 2 * c);
-        const uint32_t scB = *reinterpret_cast<const uint16_t*>(s + (size_t(e) * a.N + rB) * spr + G * 8 + 2 * c);
-        const uint8_t* rowA = smem + g * stride + G * 64 + c * 16;
-        fp4_group(rowA, rowA + 8 * stride, scA, scB, xc, two, acc);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) xc[nt][m] = xn[nt][m];
-    }
-
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) red[warp][nt][lane][i] = acc[nt][i];
-    __syncthreads();
-    if (warp == 0) {
-      float post = 1.f;
-      if (FMT == MOE_FMT_NVFP4) post = a.gscale[e] * 256.f;
+    for (int G = 0; G < GK; ++G) {
+      cp_async_wait_depth();
+      __syncwarp();  // every lane's copies of group G have landed
+      const uint8_t* sl = wsm + (G % kDepth) * a.slot_bytes;
+      uint4 xv[2][4];
+      float X[2][2];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        float v[4];
+        X[nt][0] = X[nt][1] = 0.f;
+        if ((nt == 1 && !two) || nt * 8 + g >= nvalid) {  // B column of an absent token
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float sacc = red[0][nt][lane][i];
+          for (int m = 0; m < 4; ++m) xv[nt][m] = make_uint4(0, 0, 0, 0);
+        } else {
+          const uint8_t* xr = xbuf + size_t(nt * 8 + g) * a.x_stride + G * 256 + c * 16;
 #pragma unroll
-          for (int ww = 1; ww < kWarps; ++ww) sacc += red[ww][nt][lane][i];
-          v[i] = sacc * post;
+          for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
         }
+        if (FMT != MOE_FMT_NVFP4 && !(nt == 1 && !two)) {
+          X[nt][0] = xsum[(nt * 8 + 2 * c) * GK + G];
+          X[nt][1] = xsum[(nt * 8 + 2 * c + 1) * GK + G];
+        }
+      }
+      if (FMT == MOE_FMT_W4G128) {
+        const uint8_t* wr = sl + g * 64 + c * 16;
+        w4_group(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv, two,
+                 bf16_bits_to_float(wscale[g * GK + G]), bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
+      } else if (FMT == MOE_FMT_BITPLANE8) {
+        bp_group(sl + g * 16 + c * 4, nplanes, xv, two, bt, bf16_bits_to_float(wscale[g * GK + G]),
+                 bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
+      } else {
+        const uint8_t* wr = sl + g * 64 + c * 16;
+        const uint8_t* sc = sl + kRows * 64;  // [16 rows][8 block scales]
+        const uint32_t scA = *reinterpret_cast<const uint16_t*>(sc + g * 8 + 2 * c);
+        const uint32_t scB = *reinterpret_cast<const uint16_t*>(sc + (g + 8) * 8 + 2 * c);
+        fp4_group(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), scA, scB, xv,
+                  two, acc);
+      }
+      __syncwarp();  // every lane is done with this slot before it is refilled
+      if (G + kDepth < GK) issue(G + kDepth);
+      cp_async_commit();
+    }
+    cp_async_wait_all();
+
+    // ---- epilogue: C fragment = rows g / g+8, tokens 2c, 2c+1 of each n8 tile
+    float post = 1.f;
+    if (FMT == MOE_FMT_NVFP4) post = a.gscale[e] * 256.f;
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int n = n0 + nt * 8 + 2 * c + jj;
-          if (n >= n_e) continue;
-          const size_t orow = size_t(row0 + n) * a.out_ld;
-          if (MODE == kGateUp) {
-            const float h = silu(v[jj]) * v[2 + jj];
-            const int col = 8 * blockIdx.x + g;
-            if (FMT == MOE_FMT_NVFP4)
-              static_cast<__half*>(a.out)[orow + col] = __float2half_rn(h * (1.0f / 256.f));
-            else
-              static_cast<uint16_t*>(a.out)[orow + col] = float_to_bf16_bits(h);
-          } else {
-            uint16_t* y = static_cast<uint16_t*>(a.out);
-            y[orow + kRows * blockIdx.x + g] = float_to_bf16_bits(v[jj]);
-            y[orow + kRows * blockIdx.x + g + 8] = float_to_bf16_bits(v[2 + jj]);
-          }
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int n = nt * 8 + 2 * c + jj;
+        if (n >= nvalid) continue;
+        const size_t orow = size_t(row0 + tok0 + n) * a.out_ld;
+        const float v0 = acc[nt][jj] * post, v1 = acc[nt][2 + jj] * post;
+        if (MODE == kGateUp) {
+          const float h = silu(v0) * v1;
+          const int col = 8 * rt + g;
+          if (FMT == MOE_FMT_NVFP4)
+            static_cast<__half*>(a.out)[orow + col] = __float2half_rn(h * (1.0f / 256.f));
+          else
+            static_cast<uint16_t*>(a.out)[orow + col] = float_to_bf16_bits(h);
+        } else {
+          uint16_t* y = static_cast<uint16_t*>(a.out);
+          y[orow + kRows * rt + g] = float_to_bf16_bits(v0);
+          y[orow + kRows * rt + g + 8] = float_to_bf16_bits(v1);
         }
       }
     }
-    __syncthreads();
   }
 }
 
-// x (bf16) -> fp16 * 2^-8 for the NVFP4 path (exact for |x| in [2^-6, 1.6e7]).
-__global__ void k_to_f16_scaled(const uint16_t* __restrict__ x, int64_t n, __half* __restrict__ y) {
-  const int64_t i = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) * 2;
-  if (i >= n) return;
-  const uint32_t v = *reinterpret_cast<const uint32_t*>(x + i);
-  *reinterpret_cast<__half2*>(y + i) = __floats2half2_rn(bf16_lo(v) * (1.0f / 256.f), bf16_hi(v) * (1.0f / 256.f));
-}
-
-// ---------------------------------------------------------------- launchers
+// ---------------------------------------------------------------- launch planning
 static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
-size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t /*E*/, int64_t k, moe_format_t fmt) {
-  size_t b = align256(size_t(T * k * I * 2));  // h
-  if (fmt == MOE_FMT_NVFP4) b += align256(size_t(T * H * 2));  // x as fp16
-  return b;
+size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t /*E*/, int64_t k, moe_format_t /*fmt*/) {
+  return align256(size_t(T * k * I * 2));  // h
+}
+
+template <int FMT>
+static bool plan(FfnArgs& a) {
+  const int K = a.K, GK = K / 128;
+  a.slot_bytes = slot_bytes_of<FMT>();
+  const int scale_bytes = (FMT == MOE_FMT_NVFP4) ? 0 : int(align256(size_t(kRows) * GK * 2));
+  a.warp_bytes = int(align256(size_t(kDepth) * a.slot_bytes + scale_bytes));
+  a.x_stride = stride_16B(K * 2);
+  const size_t fixed = size_t(kWarps) * a.warp_bytes + align256(size_t(kMaxTok) * GK * 4) + 256;
+  const size_t room = fixed < kSmemTarget ? kSmemTarget - fixed : 0;
+  int nx = int(room / size_t(a.x_stride));
+  nx = nx < 1 ? 1 : nx;  // wide rows: at least one token row (then one CTA per SM)
+  a.nx = nx > kMaxTok ? kMaxTok : nx;
+  size_t off = size_t(kWarps) * a.warp_bytes;
+  a.off_x = int(off);
+  off += align256(size_t(a.nx) * a.x_stride);
+  a.off_xsum = int(off);
+  off += align256(size_t(kMaxTok) * GK * 4);
+  a.off_bits = int(off);
+  off += 256;
+  return off <= 220 * 1024;
 }
 
 template <int FMT, int MODE>
-static cudaError_t launch_one(const FfnArgs& a, int tiles, int slots, cudaStream_t st) {
-  const size_t smem = ffn_smem_bytes<FMT>(a.K);
-  if (smem > 48 * 1024) {
+static cudaError_t launch_one(FfnArgs a, int slots, cudaStream_t st) {
+  if (!plan<FMT>(a)) return cudaErrorInvalidValue;
+  const size_t smem = size_t(a.off_bits) + 256;
+  // raise the kernel's dynamic shared-memory limit once per device (kept out of later
+  // calls, which may be inside a graph capture)
+  static bool raised[128] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (!raised[dev]) {
     cudaError_t err =
-        cudaFuncSetAttribute(k_ffn_gemv<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaFuncSetAttribute(k_ffn_gemv<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
     if (err != cudaSuccess) return err;
+    raised[dev] = true;
   }
-  k_ffn_gemv<FMT, MODE><<<dim3(unsigned(tiles), unsigned(slots)), 32 * kWarps, smem, st>>>(a);
+  const int TPE = (MODE == kGateUp) ? a.I / 8 : a.N / kRows;
+  k_ffn_gemv<FMT, MODE><<<dim3(unsigned((TPE + kWarps - 1) / kWarps), unsigned(slots)), kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 template <int FMT>
-static cudaError_t launch_fmt(const void* act_x, const moe_routing_t& r, const moe_experts_t& ex,
-                              const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,
-                              void* hbuf, cudaStream_t st) {
+static cudaError_t launch_fmt(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
+                              const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows, void* hbuf,
+                              cudaStream_t st) {
   const int P = T * k;
   const int slots = P < E ? P : E;
   FfnArgs a{};
@@ -460,9 +531,8 @@ static cudaError_t launch_fmt(const void* act_x, const moe_routing_t& r, const m
   a.offsets = r.expert_offsets;
   a.sorted_pair = r.sorted_pair;
   a.bits = bits;
-  a.err = device_error_word();
   // gate/up
-  a.act = act_x;
+  a.act = x;
   a.K = H;
   a.N = 2 * I;
   a.w = ex.w13;
@@ -470,7 +540,7 @@ static cudaError_t launch_fmt(const void* act_x, const moe_routing_t& r, const m
   a.gscale = ex.w13_gscale;
   a.out = hbuf;
   a.out_ld = I;
-  cudaError_t err = launch_one<FMT, kGateUp>(a, I / 8, slots, st);
+  cudaError_t err = launch_one<FMT, kGateUp>(a, slots, st);
   if (err != cudaSuccess) return err;
   // down
   a.act = hbuf;
@@ -481,27 +551,31 @@ static cudaError_t launch_fmt(const void* act_x, const moe_routing_t& r, const m
   a.gscale = ex.w2_gscale;
   a.out = y_rows;
   a.out_ld = H;
-  return launch_one<FMT, kDown>(a, H / kRows, slots, st);
+  return launch_one<FMT, kDown>(a, slots, st);
+}
+
+bool ffn_shape_supported(int64_t H, int64_t I, moe_format_t fmt) {
+  FfnArgs a{};
+  bool ok = true;
+  for (int64_t K : {H, I}) {
+    a.K = int(K);
+    ok = ok && (fmt == MOE_FMT_BITPLANE8 ? plan<MOE_FMT_BITPLANE8>(a)
+                : fmt == MOE_FMT_NVFP4   ? plan<MOE_FMT_NVFP4>(a)
+                                         : plan<MOE_FMT_W4G128>(a));
+  }
+  return ok;
 }
 
 cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
-                               const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,
-                               void* ws, cudaStream_t st) {
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  void* hbuf = w8;
+                               const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows, void* ws,
+                               cudaStream_t st) {
   switch (ex.fmt) {
     case MOE_FMT_W4G128:
-      return launch_fmt<MOE_FMT_W4G128>(x, r, ex, bits, T, H, I, E, k, y_rows, hbuf, st);
+      return launch_fmt<MOE_FMT_W4G128>(x, r, ex, bits, T, H, I, E, k, y_rows, ws, st);
     case MOE_FMT_BITPLANE8:
-      return launch_fmt<MOE_FMT_BITPLANE8>(x, r, ex, bits, T, H, I, E, k, y_rows, hbuf, st);
-    case MOE_FMT_NVFP4: {
-      __half* x16 = reinterpret_cast<__half*>(w8 + align256(size_t(T) * k * I * 2));
-      const int64_t n = int64_t(T) * H;
-      k_to_f16_scaled<<<dim3(unsigned((n / 2 + 255) / 256)), 256, 0, st>>>(x, n, x16);
-      cudaError_t err = cudaGetLastError();
-      if (err != cudaSuccess) return err;
-      return launch_fmt<MOE_FMT_NVFP4>(x16, r, ex, bits, T, H, I, E, k, y_rows, hbuf, st);
-    }
+      return launch_fmt<MOE_FMT_BITPLANE8>(x, r, ex, bits, T, H, I, E, k, y_rows, ws, st);
+    case MOE_FMT_NVFP4:
+      return launch_fmt<MOE_FMT_NVFP4>(x, r, ex, bits, T, H, I, E, k, y_rows, ws, st);
   }
   return cudaErrorInvalidValue;
 }

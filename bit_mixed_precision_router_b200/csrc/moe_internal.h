@@ -24,6 +24,7 @@ cudaError_t launch_select_bits(const float* w, int64_t n, const float thr[3], co
                                uint8_t* bits, cudaStream_t st);
 
 // Grouped FFN.
+bool ffn_shape_supported(int64_t H, int64_t I, moe_format_t fmt);
 size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, moe_format_t fmt);
 cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
                                const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,

@@ -87,7 +87,7 @@ def test_ffn_and_combine_validation(lib):
     assert call(4, 2048, 1024, 64, 8, ws=None) == WS
     assert call(4, 2048, 1024, 64, 8, wsb=1024) == WS
     assert call(0, 2048, 1024, 64, 8, ws=None, wsb=0) == OK
-    assert call(4, 65536, 1024, 64, 8) == SHAPE  # weight tile would not fit in shared memory
+    assert call(4, 131072, 1024, 64, 8) == SHAPE  # larger than the supported hidden size
     ex.fmt = 1
     assert call(4, 2048, 1024, 64, 8) == INVALID  # bitplanes need the bits array
     ex.fmt = 2
@@ -95,7 +95,6 @@ def test_ffn_and_combine_validation(lib):
     ex.fmt = 7
     assert call(4, 2048, 1024, 64, 8) == INVALID
     assert lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 0) >= 16 * 8 * 1024 * 2
-    assert lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 2) > lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 0)
     c = lambda T, H, k, res=None: lib.moe_combine(A, ctypes.byref(r), res, T, H, k, A, None)
     assert c(4, 2044, 8) == SHAPE
     assert c(4, 2048, 0) == INVALID
