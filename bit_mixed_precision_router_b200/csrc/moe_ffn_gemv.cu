@@ -75,18 +75,22 @@ MOE_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: 
 // of tile nt; X[nt][j] the group sum of the activations of token 2c+j of tile nt.
 
 // INT4: nibbles j and j+4 of a word become one bf16x2 of (128 + u) with one shift and one
-// LOP3; the activations were paired (j, j+4) when staged.  The MMA sums (q + 136) * x;
-// 136 * sum(x) is removed with the staged group sums.
-MOE_DEVICE void w4_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], bool two, float sa, float sb,
-                         const float (&X)[2][2], float (&acc)[2][4]) {
+// LOP3; the activations were paired (j, j+4) when staged.  The MMA sums (q + 136) * x onto
+// an accumulator seeded with -136 * sum(x) (the staged group sums), so after the group it
+// holds sum q * x and one FMA applies the row's scale.
+template <bool TWO>
+MOE_DEVICE void w4_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa, float sb, const float (&X)[2][2],
+                         float (&acc)[2][4]) {
   const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
   const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
   constexpr uint32_t kMagic = 0x43004300u;  // bf16 (128, 128)
-  float t0[2][4], t1[2][4];
+  constexpr int NT = TWO ? 2 : 1;
+  float t[2][4];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) t0[nt][i] = t1[nt][i] = 0.f;
+  for (int nt = 0; nt < NT; ++nt) {
+    t[nt][0] = t[nt][2] = -136.f * X[nt][0];
+    t[nt][1] = t[nt][3] = -136.f * X[nt][1];
+  }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     uint32_t pa[4], pb[4];
@@ -96,21 +100,18 @@ MOE_DEVICE void w4_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], bool two, 
       pb[j] = ((wb_[m] >> (4 * j)) & 0x000F000Fu) | kMagic;
     }
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      if (nt == 1 && !two) break;
+    for (int nt = 0; nt < NT; ++nt) {
       const uint4 xx = xv[nt][m];
-      float(&t)[4] = (m & 1) ? t1[nt] : t0[nt];
-      mma_bf16(t, pa[0], pb[0], pa[1], pb[1], xx.x, xx.y);
-      mma_bf16(t, pa[2], pb[2], pa[3], pb[3], xx.z, xx.w);
+      mma_bf16(t[nt], pa[0], pb[0], pa[1], pb[1], xx.x, xx.y);
+      mma_bf16(t[nt], pa[2], pb[2], pa[3], pb[3], xx.z, xx.w);
     }
   }
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    const float c0 = 136.f * X[nt][0], c1 = 136.f * X[nt][1];
-    acc[nt][0] = fmaf(sa, (t0[nt][0] + t1[nt][0]) - c0, acc[nt][0]);
-    acc[nt][1] = fmaf(sa, (t0[nt][1] + t1[nt][1]) - c1, acc[nt][1]);
-    acc[nt][2] = fmaf(sb, (t0[nt][2] + t1[nt][2]) - c0, acc[nt][2]);
-    acc[nt][3] = fmaf(sb, (t0[nt][3] + t1[nt][3]) - c1, acc[nt][3]);
+  for (int nt = 0; nt < NT; ++nt) {
+    acc[nt][0] = fmaf(sa, t[nt][0], acc[nt][0]);
+    acc[nt][1] = fmaf(sa, t[nt][1], acc[nt][1]);
+    acc[nt][2] = fmaf(sb, t[nt][2], acc[nt][2]);
+    acc[nt][3] = fmaf(sb, t[nt][3], acc[nt][3]);
   }
 }
 
@@ -127,8 +128,10 @@ MOE_DEVICE uint32_t bit_pair(uint32_t w, int j) {
 MOE_DEVICE float plane_coef_x(int b) { return (b >= 8) ? -383.f : float(3 * (1 << (7 - b)) - 384); }
 
 // pl: the thread's word of plane 0, row g; planes are 16 rows x 16 bytes apart.
-MOE_DEVICE void bp_group(const uint8_t* pl, int nplanes, const uint4 (&xv)[2][4], bool two, const int (&bt)[2][2],
-                         float sa, float sb, const float (&X)[2][2], float (&acc)[2][4]) {
+template <bool TWO>
+MOE_DEVICE void bp_group(const uint8_t* pl, int nplanes, const uint4 (&xv)[2][4], const int (&bt)[2][2], float sa,
+                         float sb, const float (&X)[2][2], float (&acc)[2][4]) {
+  constexpr bool two = TWO;
   float grp[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
@@ -192,8 +195,10 @@ MOE_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {
   return d;
 }
 
-MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const uint4 (&xv)[2][4], bool two,
+template <bool TWO>
+MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const uint4 (&xv)[2][4],
                           float (&acc)[2][4]) {
+  constexpr bool two = TWO;
   const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
   const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
   // words 0,1 -> block 2c (byte 0 of sc), words 2,3 -> block 2c+1 (byte 1)
@@ -214,6 +219,57 @@ MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const 
       mma_f16(acc[nt], ha[0], hb[0], ha[1], hb[1], xx.x, xx.y);
       mma_f16(acc[nt], ha[2], hb[2], ha[3], hb[3], xx.z, xx.w);
     }
+  }
+}
+
+// ---------------------------------------------------------------- one unit
+// Streams the warp's unit: for G = 0 .. GK-1, waits for group G's slot, computes it
+// against the staged activations of one (TWO = false) or two n8 token tiles, and refills
+// the slot with group G + kDepth.
+template <int FMT, bool TWO, class Issue>
+MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t* wscale, const uint8_t* xbuf,
+                            const float* xsum, int GK, int g, int c, int nvalid, int nplanes, const int (&bt)[2][2],
+                            Issue&& issue, float (&acc)[2][4]) {
+  constexpr int NT = TWO ? 2 : 1;
+  for (int G = 0; G < GK; ++G) {
+    cp_async_wait_depth();
+    __syncwarp();  // every lane's copies of group G have landed
+    const uint8_t* sl = wsm + (G % kDepth) * a.slot_bytes;
+    uint4 xv[2][4];
+    float X[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (nt * 8 + g >= nvalid) {  // B column of an absent token
+#pragma unroll
+        for (int m = 0; m < 4; ++m) xv[nt][m] = make_uint4(0, 0, 0, 0);
+      } else {
+        const uint8_t* xr = xbuf + size_t(nt * 8 + g) * a.x_stride + G * 256 + c * 16;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
+      }
+      if (FMT != MOE_FMT_NVFP4) {  // group sums of C columns 2c, 2c+1 (kMaxTok rows staged)
+        X[nt][0] = xsum[(nt * 8 + 2 * c) * GK + G];
+        X[nt][1] = xsum[(nt * 8 + 2 * c + 1) * GK + G];
+      }
+    }
+    if (FMT == MOE_FMT_W4G128) {
+      const uint8_t* wr = sl + g * 64 + c * 16;
+      w4_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
+                    bf16_bits_to_float(wscale[g * GK + G]), bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
+    } else if (FMT == MOE_FMT_BITPLANE8) {
+      bp_group<TWO>(sl + g * 16 + c * 4, nplanes, xv, bt, bf16_bits_to_float(wscale[g * GK + G]),
+                    bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
+    } else {
+      const uint8_t* wr = sl + g * 64 + c * 16;
+      const uint8_t* sc = sl + kRows * 64;  // [16 rows][8 block scales]
+      const uint32_t scA = *reinterpret_cast<const uint16_t*>(sc + g * 8 + 2 * c);
+      const uint32_t scB = *reinterpret_cast<const uint16_t*>(sc + (g + 8) * 8 + 2 * c);
+      fp4_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), scA, scB,
+                     xv, acc);
+    }
+    __syncwarp();  // every lane is done with this slot before it is refilled
+    if (G + kDepth < GK) issue(G + kDepth);
+    cp_async_commit();
   }
 }
 
@@ -397,47 +453,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    for (int G = 0; G < GK; ++G) {
-      cp_async_wait_depth();
-      __syncwarp();  // every lane's copies of group G have landed
-      const uint8_t* sl = wsm + (G % kDepth) * a.slot_bytes;
-      uint4 xv[2][4];
-      float X[2][2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        X[nt][0] = X[nt][1] = 0.f;
-        if ((nt == 1 && !two) || nt * 8 + g >= nvalid) {  // B column of an absent token
-#pragma unroll
-          for (int m = 0; m < 4; ++m) xv[nt][m] = make_uint4(0, 0, 0, 0);
-        } else {
-          const uint8_t* xr = xbuf + size_t(nt * 8 + g) * a.x_stride + G * 256 + c * 16;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
-        }
-        if (FMT != MOE_FMT_NVFP4 && !(nt == 1 && !two)) {
-          X[nt][0] = xsum[(nt * 8 + 2 * c) * GK + G];
-          X[nt][1] = xsum[(nt * 8 + 2 * c + 1) * GK + G];
-        }
-      }
-      if (FMT == MOE_FMT_W4G128) {
-        const uint8_t* wr = sl + g * 64 + c * 16;
-        w4_group(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv, two,
-                 bf16_bits_to_float(wscale[g * GK + G]), bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
-      } else if (FMT == MOE_FMT_BITPLANE8) {
-        bp_group(sl + g * 16 + c * 4, nplanes, xv, two, bt, bf16_bits_to_float(wscale[g * GK + G]),
-                 bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
-      } else {
-        const uint8_t* wr = sl + g * 64 + c * 16;
-        const uint8_t* sc = sl + kRows * 64;  // [16 rows][8 block scales]
-        const uint32_t scA = *reinterpret_cast<const uint16_t*>(sc + g * 8 + 2 * c);
-        const uint32_t scB = *reinterpret_cast<const uint16_t*>(sc + (g + 8) * 8 + 2 * c);
-        fp4_group(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), scA, scB, xv,
-                  two, acc);
-      }
-      __syncwarp();  // every lane is done with this slot before it is refilled
-      if (G + kDepth < GK) issue(G + kDepth);
-      cp_async_commit();
-    }
+    if (two)
+      stream_unit<FMT, true>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, nplanes, bt, issue, acc);
+    else
+      stream_unit<FMT, false>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, nplanes, bt, issue, acc);
     cp_async_wait_all();
 
     // ---- epilogue: C fragment = rows g / g+8, tokens 2c, 2c+1 of each n8 tile
