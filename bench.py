@@ -193,8 +193,7 @@ class DecodeStack:
         del tmp13, tmp2
         B = batch
         self.routing = moe.Routing.empty(B, E, K_TOP, device)
-        self.route_ws = torch.empty(max(moe.moe_route_workspace_bytes(B, E, K_TOP), 16), dtype=torch.uint8,
-                                    device=device)
+        self.route_ws = moe.moe_route_workspace(B, E, K_TOP, device)
         self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(B, H, I, E, K_TOP, moe.FMT_W4G128), 16),
                                   dtype=torch.uint8, device=device)
         self.y_rows = torch.empty((B * K_TOP, H), dtype=torch.bfloat16, device=device)
@@ -222,7 +221,10 @@ class DecodeStack:
 
     @property
     def kernels_per_step(self):
-        return self.L * 5  # logits, top-k+permute, gate/up, down, combine
+        # router: one launch for up to 16 tokens whose bf16 rows fit 64 KiB, else logits,
+        # top-k and permutation; then gate/up, down and combine
+        route = 1 if (self.B <= 16 and self.B * H * 2 <= 64 * 1024) else 3
+        return self.L * (route + 3)
 
 
 def run_gpu(args, rank, world, local):

@@ -179,14 +179,19 @@ def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:
     return int(load().moe_route_workspace_bytes(T, E, k))
 
 
+def moe_route_workspace(T: int, E: int, k: int, device) -> torch.Tensor:
+    """A zero-filled router workspace for up to (T, E, k); reusable across calls
+    (each call leaves its completion counter at zero)."""
+    return torch.zeros(max(moe_route_workspace_bytes(T, E, k), 16), dtype=torch.uint8, device=device)
+
+
 def moe_route_topk(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | None, k: int,
                    out: Routing | None = None, workspace: torch.Tensor | None = None, stream=None) -> Routing:
     T, H = x.shape
     E = w_router.shape[0]
     out = Routing.empty(T, E, k, x.device) if out is None else out
-    need = moe_route_workspace_bytes(T, E, k)
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+        workspace = moe_route_workspace(T, E, k, x.device)
     rc = out.c()
     _call("moe_route_topk", _p(_bits(x)), _p(_bits(w_router)), _p(bias), T, H, E, k, ctypes.byref(rc),
           _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))

@@ -84,53 +84,60 @@ __global__ void __launch_bounds__(32 * WT * WE) k_router_logits(const uint16_t* 
 }
 
 // ---------------------------------------------------------------- top-k
-struct Cand {
-  float v;
-  int i;
-};
-MOE_DEVICE bool better(Cand a, Cand b) { return a.v > b.v || (a.v == b.v && a.i < b.i); }
+// Order-preserving unsigned key of a logit: larger logit -> larger key.  NaN ranks
+// with -inf; -0 is folded into +0 so that equal logits tie by expert id.  Key 0 is
+// below every logit and marks "no candidate".
+MOE_DEVICE uint32_t order_key(float f) {
+  if (f != f) f = -INFINITY;
+  if (f == 0.f) f = 0.f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+MOE_DEVICE float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
 
-// One warp selects token t's top-k from logits[t][0..E) and writes ids and
-// softmax weights; also returns the ids to the caller's lanes (lane j holds slot j).
-MOE_DEVICE int warp_topk(const float* __restrict__ lg, int E, int k, int t, int32_t* __restrict__ ids,
-                         float* __restrict__ w) {
+// One warp selects token t's top-k from logits[t][0..E), E <= 32 * NV, and writes ids
+// and softmax weights; also returns the ids to the caller's lanes (lane j holds slot
+// j).  Lane L holds experts q*32 + L.  Each round takes the warp maximum of the lanes'
+// best keys, then the lowest expert id among the lanes that hold that key.
+template <int NV>
+MOE_DEVICE int warp_topk_nv(const float* lg, int E, int k, int t, int32_t* __restrict__ ids,
+                            float* __restrict__ w) {
   const int lane = threadIdx.x & 31;
-  constexpr int kMaxPerLane = MOE_MAX_EXPERTS / 32;
-  float val[kMaxPerLane];
-  uint32_t taken = 0;
+  uint32_t key[NV];
 #pragma unroll
-  for (int q = 0; q < kMaxPerLane; ++q) {
+  for (int q = 0; q < NV; ++q) {
     const int e = q * 32 + lane;
-    float f = (e < E) ? lg[e] : -INFINITY;
-    if (f != f) f = -INFINITY;  // NaN ranks last
-    val[q] = f;
+    key[q] = (e < E) ? order_key(__ldcg(lg + e)) : 0u;
   }
-  Cand mine{-INFINITY, 0x7fffffff};
+  uint32_t my_key = 0;
   int my_id = -1;
   for (int j = 0; j < k; ++j) {
-    Cand best{-INFINITY, 0x7fffffff};
+    uint32_t bk = 0;
+    int bq = 0;
 #pragma unroll
-    for (int q = 0; q < kMaxPerLane; ++q) {
-      const int e = q * 32 + lane;
-      if (e < E && !((taken >> q) & 1u)) {
-        const Cand c{val[q], e};
-        if (better(c, best)) best = c;
+    for (int q = 0; q < NV; ++q)
+      if (key[q] > bk) {  // strict: the lowest expert id among this lane's equal keys
+        bk = key[q];
+        bq = q;
       }
-    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t id = __reduce_min_sync(0xffffffffu, bk == m ? uint32_t(bq * 32 + lane) : 0xffffffffu);
+    if (int(id & 31u) == lane) {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      Cand o{__shfl_xor_sync(0xffffffffu, best.v, off), __shfl_xor_sync(0xffffffffu, best.i, off)};
-      if (better(o, best)) best = o;
+      for (int q = 0; q < NV; ++q)
+        if (q == int(id >> 5)) key[q] = 0u;
     }
-    if ((best.i & 31) == lane) taken |= 1u << (best.i >> 5);
     if (lane == j) {
-      mine = best;
-      my_id = best.i;
+      my_key = m;
+      my_id = int(id);
     }
   }
   // softmax over the k selected, relative to the largest (slot 0)
-  const float l0 = __shfl_sync(0xffffffffu, mine.v, 0);
-  const float ex = (lane < k) ? expf(mine.v - l0) : 0.f;
+  const float mine = key_value(my_key);
+  const float l0 = __shfl_sync(0xffffffffu, mine, 0);
+  const float ex = (lane < k) ? expf(mine - l0) : 0.f;
   float sum = 0.f;
   for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);
   if (lane < k) {
@@ -138,6 +145,16 @@ MOE_DEVICE int warp_topk(const float* __restrict__ lg, int E, int k, int t, int3
     w[size_t(t) * k + lane] = __fdiv_rn(ex, sum);
   }
   return my_id;
+}
+
+MOE_DEVICE int warp_topk(const float* lg, int E, int k, int t, int32_t* __restrict__ ids, float* __restrict__ w) {
+  static_assert(MOE_MAX_EXPERTS <= 1024, "warp_topk holds at most 32 logits per lane");
+  if (E <= 32) return warp_topk_nv<1>(lg, E, k, t, ids, w);
+  if (E <= 64) return warp_topk_nv<2>(lg, E, k, t, ids, w);
+  if (E <= 128) return warp_topk_nv<4>(lg, E, k, t, ids, w);
+  if (E <= 256) return warp_topk_nv<8>(lg, E, k, t, ids, w);
+  if (E <= 512) return warp_topk_nv<16>(lg, E, k, t, ids, w);
+  return warp_topk_nv<32>(lg, E, k, t, ids, w);
 }
 
 __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ ids,
@@ -148,71 +165,64 @@ __global__ void k_topk(const float* __restrict__ logits, int T, int E, int k, in
 }
 
 // ---------------------------------------------------------------- permutation
-// Block-wide exclusive scan of one value per thread (blockDim.x == 1024).
-MOE_DEVICE int block_exclusive_scan(int v, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int inc = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, inc, off);
-    if (lane >= off) inc += n;
-  }
-  if (lane == 31) warp_sums[warp] = inc;
+// Stable counting sort of P = T*k pairs by expert, by one CTA of NW = blockDim.x/32
+// warps.  Warp w owns pairs [w*P/NW, (w+1)*P/NW); `cnt` is [NW][E] ints and `tot` [E]
+// ints of shared memory.  Writes expert_offsets, expert_list, sorted_pair, pair_to_row.
+MOE_DEVICE void permute_block(const int32_t* ids, int P, int E, int* cnt, int* tot, const moe_routing_t& out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, NW = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < NW * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
-  if (warp == 0) {
-    int s = warp_sums[lane];
-    int si = s;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, si, off);
-      if (lane >= off) si += n;
-    }
-    warp_sums[lane] = si - s;  // exclusive prefix of warp totals
-    if (lane == 31) *total = si;
-  }
-  __syncthreads();
-  return warp_sums[warp] + inc - v;
-}
-
-// Stable counting sort of P = T*k pairs by expert.  One CTA of 1024 threads.
-// Warp w owns pairs [w*P/32, (w+1)*P/32); cnt is [32][E] ints of shared memory.
-MOE_DEVICE void permute_block(const int32_t* ids, int P, int E, int* cnt, int* scratch,
-                              const moe_routing_t& out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < 32 * E; i += 1024) cnt[i] = 0;
-  __syncthreads();
-  const int beg = int((int64_t(warp) * P) / 32), end = int((int64_t(warp + 1) * P) / 32);
+  const int beg = int((int64_t(warp) * P) / NW), end = int((int64_t(warp + 1) * P) / NW);
   for (int p = beg + lane; p < end; p += 32) atomicAdd(&cnt[warp * E + ids[p]], 1);
   __syncthreads();
-  // per expert: column prefix over warps, then the scan over experts
-  int* warp_sums = scratch;   // [32]
-  int* total_out = scratch + 32;
-  int* n_active = scratch + 33;
-  for (int eb = 0; eb < E; eb += 1024) {
-    // E <= 1024, so this loop runs once; kept explicit for clarity
-    const int e = eb + threadIdx.x;
-    int tot = 0;
-    if (e < E)
-      for (int ww = 0; ww < 32; ++ww) tot += cnt[ww * E + e];
-    const int off = block_exclusive_scan(tot, warp_sums, total_out);
-    const int flag = (e < E && tot > 0) ? 1 : 0;
-    const int pos = block_exclusive_scan(flag, warp_sums, n_active);
-    if (e < E) {
-      out.expert_offsets[e] = off;
-      if (flag) out.expert_list[1 + pos] = e;
-      int run = off;
-      for (int ww = 0; ww < 32; ++ww) {
-        const int c = cnt[ww * E + e];
-        cnt[ww * E + e] = run;
-        run += c;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int t = 0;
+    for (int w = 0; w < NW; ++w) t += cnt[w * E + e];
+    tot[e] = t;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive prefix over experts and the ordered list of active experts; lane L owns
+    // the contiguous range [L*per, (L+1)*per)
+    const int per = (E + 31) / 32;
+    const int b = min(E, lane * per), en = min(E, b + per);
+    int sum = 0, act = 0;
+    for (int e = b; e < en; ++e) {
+      sum += tot[e];
+      act += tot[e] > 0;
+    }
+    int isum = sum, iact = act;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v1 = __shfl_up_sync(0xffffffffu, isum, off), v2 = __shfl_up_sync(0xffffffffu, iact, off);
+      if (lane >= off) {
+        isum += v1;
+        iact += v2;
       }
+    }
+    int run = isum - sum, pos = iact - act;
+    for (int e = b; e < en; ++e) {
+      const int t = tot[e];
+      out.expert_offsets[e] = run;
+      if (t > 0) out.expert_list[1 + pos++] = e;
+      tot[e] = run;
+      run += t;
+    }
+    if (lane == 31) {
+      out.expert_offsets[E] = P;
+      out.expert_list[0] = iact;
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    out.expert_offsets[E] = P;
-    out.expert_list[0] = *n_active;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = tot[e];
+    for (int w = 0; w < NW; ++w) {
+      const int c = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += c;
+    }
   }
+  __syncthreads();
   // stable scatter: walk each warp's range in order, 32 pairs at a time
   for (int base = beg; base < end; base += 32) {
     const int p = base + lane;
@@ -236,23 +246,111 @@ MOE_DEVICE void permute_block(const int32_t* ids, int P, int E, int* cnt, int* s
 __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ ids, int P, int E,
                                                   moe_routing_t out) {
   extern __shared__ int smem_i[];
-  __shared__ int scratch[40];
-  permute_block(ids, P, E, smem_i, scratch, out);
+  permute_block(ids, P, E, smem_i, smem_i + 32 * E, out);
 }
 
-// Small batches: top-k of every token and the permutation in one CTA.
-__global__ void __launch_bounds__(1024) k_topk_permute_small(const float* __restrict__ logits, int T, int E,
-                                                             int k, moe_routing_t out) {
-  extern __shared__ int smem_i[];
-  __shared__ int scratch[40];
-  int* ids_s = smem_i + 32 * E;  // [T*k]
+// ---------------------------------------------------------------- small batches, fused
+// One launch for few tokens: CTA b computes the logits of experts 8b .. 8b+7 for every
+// token (warp = expert; the tokens are staged once in shared memory; the router row's
+// chunks are loaded before any FMA), in the same fixed order as k_router_logits.  The
+// last CTA to finish (ticket counter, reset to 0 by that CTA) reads all logits back,
+// selects every token's top-k and builds the permutation.
+constexpr int kFusedMaxT = 16;
+constexpr int kFusedWarps = 8;
+
+__global__ void __launch_bounds__(32 * kFusedWarps) k_route_fused(const uint16_t* __restrict__ x,
+                                                                 const uint16_t* __restrict__ wr,
+                                                                 const float* __restrict__ bias, int T, int H, int E,
+                                                                 int k, float* logits, unsigned* ticket,
+                                                                 moe_routing_t out) {
+  extern __shared__ __align__(16) uint8_t smem_u8[];
+  __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < T; t += 32) {
+  const int e = blockIdx.x * kFusedWarps + warp;
+  const uint16_t* wrow = wr + size_t(e < E ? e : 0) * H;
+  const int J = H / 256;
+  // the first eight 256-wide chunks of this warp's router row are requested before
+  // the tokens are staged, so the two memory latencies overlap
+  uint4 wv[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    wv[q] = (e < E && q < J) ? ldg_nc_v4(wrow + 256 * q + 8 * lane) : make_uint4(0, 0, 0, 0);
+  // stage the tokens, four 16-byte loads in flight per thread
+  {
+    const int n16 = T * H / 8;
+    const uint4* xs = reinterpret_cast<const uint4*>(x);
+    uint4* xd = reinterpret_cast<uint4*>(smem_u8);
+    for (int i0 = threadIdx.x; i0 < n16; i0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) v[u] = xs[i];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) xd[i] = v[u];
+      }
+    }
+  }
+  __syncthreads();
+  if (e < E) {
+    float acc[kFusedMaxT];
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; ++t) acc[t] = 0.f;
+    for (int j0 = 0; j0 < J; j0 += 8) {
+      if (j0 > 0) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          wv[q] = (j0 + q < J) ? ldg_nc_v4(wrow + 256 * (j0 + q) + 8 * lane) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (j0 + q >= J) break;
+        const uint32_t wu[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
+#pragma unroll
+        for (int t = 0; t < kFusedMaxT; ++t) {
+          if (t >= T) break;
+          const uint4 xv = *reinterpret_cast<const uint4*>(smem_u8 + (size_t(t) * H + 256 * (j0 + q) + 8 * lane) * 2);
+          const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float xf = (i & 1) ? bf16_hi(xu[i >> 1]) : bf16_lo(xu[i >> 1]);
+            const float wf = (i & 1) ? bf16_hi(wu[i >> 1]) : bf16_lo(wu[i >> 1]);
+            acc[t] = fmaf(xf, wf, acc[t]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; ++t) {
+      if (t >= T) break;
+      float v = acc[t];
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+      if (lane == 0) logits[size_t(t) * E + e] = bias ? v + bias[e] : v;
+    }
+  }
+  // last CTA: top-k and permutation
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int* ids_s = reinterpret_cast<int*>(smem_u8);  // the staged tokens are no longer needed
+  for (int t = warp; t < T; t += kFusedWarps) {
     const int id = warp_topk(logits + size_t(t) * E, E, k, t, out.topk_ids, out.topk_w);
     if (lane < k) ids_s[t * k + lane] = id;
   }
   __syncthreads();
-  permute_block(ids_s, T * k, E, smem_i, scratch, out);
+  const int P = T * k;
+  int* cnt = ids_s + ((P + 3) & ~3);
+  permute_block(ids_s, P, E, cnt, cnt + kFusedWarps * E, out);
+  if (threadIdx.x == 0) *ticket = 0u;
 }
 
 __global__ void k_select_bits(const float* __restrict__ w, int64_t n, float t0, float t1, float t2, uint8_t c0,
@@ -264,15 +362,40 @@ __global__ void k_select_bits(const float* __restrict__ w, int64_t n, float t0, 
 }
 
 // ---------------------------------------------------------------- launchers
-constexpr int kSmallT = 64;
+static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
-size_t route_workspace_bytes(int64_t T, int64_t E, int64_t /*k*/) {
-  return size_t(((T * E * 4) + 255) / 256 * 256);
+// fp32 logits [T][E], then one 32-bit ticket counter (must start at 0; left at 0).
+size_t route_workspace_bytes(int64_t T, int64_t E, int64_t /*k*/) { return align256(size_t(T * E * 4)) + 256; }
+
+static bool use_fused(int T, int H, int E, int k) {
+  const size_t stage = size_t(T) * H * 2;
+  const size_t perm = size_t(((T * k + 3) & ~3) + kFusedWarps * E + E) * 4;
+  return T <= kFusedMaxT && stage <= 64 * 1024 && perm <= 64 * 1024;
 }
 
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
                          const moe_routing_t& out, void* ws, cudaStream_t st) {
   float* logits = static_cast<float*>(ws);
+  unsigned* ticket = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + align256(size_t(T) * E * 4));
+  cudaError_t err;
+  if (use_fused(T, H, E, k)) {
+    const size_t stage = size_t(T) * H * 2;
+    const size_t perm = size_t(((T * k + 3) & ~3) + kFusedWarps * E + E) * 4;
+    const size_t smem = stage > perm ? stage : perm;
+    if (smem > 48 * 1024) {
+      static bool raised[128] = {};
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (dev >= 0 && dev < 128 && !raised[dev]) {
+        err = cudaFuncSetAttribute(k_route_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+        if (err != cudaSuccess) return err;
+        raised[dev] = true;
+      }
+    }
+    k_route_fused<<<dim3(unsigned((E + kFusedWarps - 1) / kFusedWarps)), 32 * kFusedWarps, smem, st>>>(
+        x, wr, bias, T, H, E, k, logits, ticket, out);
+    return cudaGetLastError();
+  }
   if (T >= 256) {
     constexpr int WT = 4, WE = 4;
     dim3 grid((T + WT * kTileT - 1) / (WT * kTileT), (E + WE * kTileE - 1) / (WE * kTileE));
@@ -281,21 +404,11 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
     dim3 grid((T + kTileT - 1) / kTileT, (E + kTileE - 1) / kTileE);
     k_router_logits<1, 1><<<grid, 32, 0, st>>>(x, wr, bias, T, H, E, logits);
   }
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int P = T * k;
-  if (T <= kSmallT) {
-    const size_t smem = size_t(32 * E + P) * sizeof(int);
-    if (smem > 48 * 1024) {
-      err = cudaFuncSetAttribute(k_topk_permute_small, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      if (err != cudaSuccess) return err;
-    }
-    k_topk_permute_small<<<1, 1024, smem, st>>>(logits, T, E, k, out);
-    return cudaGetLastError();
-  }
   k_topk<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, out.topk_ids, out.topk_w);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const size_t smem = size_t(32 * E) * sizeof(int);
+  const size_t smem = size_t(33 * E) * sizeof(int);
   if (smem > 48 * 1024) {
     err = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (err != cudaSuccess) return err;

@@ -10,12 +10,16 @@
 // library image instead of a caller-provided workspace.
 //
 // Limits and sharing:
-//   - the array holds kMaxLogits = MOE_NOALLOC_MAX_LOGITS floats (256 KiB); a call
-//     with T * E above that is rejected with MOE_ERR_UNSUPPORTED_SHAPE;
+//   - the array holds kMaxLogits = MOE_NOALLOC_MAX_LOGITS floats (256 KiB) followed
+//     by 256 bytes for the router's completion counter; a call with T * E above
+//     kMaxLogits is rejected with MOE_ERR_UNSUPPORTED_SHAPE;
 //   - every GPU that loads the library holds the array until the process exits;
 //   - all calls share it: two calls whose kernels overlap on the same GPU (for
 //     example on two streams) race on it and give undefined routing;
-//   - nothing in it needs clearing: each call writes every logit it later reads.
+//   - the logits need no clearing (each call writes every logit it later reads); the
+//     counter, which moe_route_topk expects at zero in the 256 bytes after the
+//     logits, starts at zero because device variables are zero-initialised when the
+//     module loads, and every call leaves it at zero.
 // Set-up: the first call on a device looks up the array's device address with
 // cudaGetSymbolAddress (the host-side name is only a stand-in, never a device
 // address) while that device is current, and caches it per device.  Make that
@@ -29,7 +33,7 @@ namespace {
 
 constexpr int64_t kMaxLogits = MOE_NOALLOC_MAX_LOGITS;
 
-static __device__ __align__(256) float g_route_logits_scratch[kMaxLogits];
+static __device__ __align__(256) float g_route_logits_scratch[kMaxLogits + 64];
 
 // Device address of g_route_logits_scratch on the current device, or nullptr.
 float* scratch_on_current_device() {

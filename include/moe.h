@@ -158,8 +158,13 @@ size_t moe_route_workspace_bytes(int64_t T, int64_t E, int64_t k);
  * over the k chosen.  Permutation: stable counting sort of the pairs by expert.
  *   x bf16 [T][H];  w_router bf16 [E][H];  bias fp32 [E] or NULL;  out: see moe_routing_t.
  * Requires H % 256 == 0, 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= min(E, MOE_MAX_TOPK),
- * T >= 0; workspace >= moe_route_workspace_bytes(T, E, k) (contents need not be
- * initialised; overwritten).  Ids and permutation are deterministic. */
+ * T >= 0; workspace >= moe_route_workspace_bytes(T, E, k).  Workspace contents: the
+ * last 256 bytes of the moe_route_workspace_bytes(T, E, k) region hold a completion
+ * counter that must be zero before the first call that uses this workspace (allocate
+ * it zero-filled once, e.g. cudaMemset); every call leaves it zero again, so the same
+ * workspace serves any number of later calls; the rest is scratch, overwritten.
+ * Calls whose kernels overlap on one workspace race on it.  Ids and permutation are
+ * deterministic. */
 moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const float* bias,
                             int64_t T, int64_t H, int64_t E, int64_t k,
                             const moe_routing_t* out, void* workspace, size_t workspace_bytes,
@@ -174,8 +179,9 @@ moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const f
  * that passes just inputs and outputs, or code running while a stream is captured
  * into a CUDA graph in global mode, where cudaMalloc is not allowed.
  * Same computation, arguments, results and errors as moe_route_topk, except that
- * the fp32 logits scratch is a fixed device array inside the library (256 KiB per
- * GPU that loads the library, held until exit):
+ * the fp32 logits scratch and the completion counter are a fixed device array inside
+ * the library (256 KiB + 256 bytes per GPU that loads the library, held until exit;
+ * the counter is zero when the library loads and every call leaves it zero):
  *   - T * E must be <= MOE_NOALLOC_MAX_LOGITS, else MOE_ERR_UNSUPPORTED_SHAPE;
  *   - the library allocates nothing and frees nothing during the call;
  *   - all calls share the array: calls whose kernels overlap on one GPU (e.g. on two

@@ -80,6 +80,11 @@ ROUTE_CASES = [
     (40, 256, 1024, 32, "normal", False),   # largest E and k
     (3, 256, 1, 1, "normal", False),        # a single expert
     (33, 256, 5, 5, "normal", False),       # k = E: every expert for every token
+    # single-launch path for few tokens (T <= 16, staged tokens <= 64 KiB)
+    (4, 7168, 256, 8, "uniform", False),    # wide hidden size, 56 KiB of staged tokens
+    (13, 512, 37, 6, "normal", True),       # E not a multiple of the 8 experts per CTA
+    (16, 256, 1024, 32, "normal", False),   # largest E and k with the last-CTA permutation
+    (9, 7168, 256, 8, "uniform", False),    # too many staged bytes: the multi-launch path
 ]
 
 
@@ -105,6 +110,21 @@ def test_route_topk_bitexact(moe, cuda_device, T, H, E, k, router, zipf):
     el = out.expert_list.cpu().numpy()
     act = np.nonzero(np.diff(offsets) > 0)[0]
     assert el[0] == act.size and np.array_equal(el[1:1 + act.size], act)
+
+
+@pytest.mark.parametrize("T,H,E,k", [(8, 2048, 64, 8), (1, 256, 8, 2), (100, 512, 64, 8)])
+def test_route_workspace_reuse(moe, cuda_device, T, H, E, k):
+    # one workspace for several calls: the completion counter is left at zero each time
+    ws = moe.moe_route_workspace(T, E, k, "cuda")
+    out = moe.Routing.empty(T, E, k)
+    for rep in range(3):
+        L = make_layer(900 + rep, T, H, 128, E, k, with_experts=False)
+        moe.moe_route_topk(dev_bf16(L.x), dev_bf16(L.wr), None, k, out=out, workspace=ws)
+        ids, w = topk_softmax(router_logits(L.x, L.wr, None), k)
+        offsets, sp, p2r = permute(ids, E)
+        assert np.array_equal(out.topk_ids.cpu().numpy().reshape(T, k), ids)
+        assert np.array_equal(out.sorted_pair.cpu().numpy(), sp)
+        assert not ws[-256:].any().item()
 
 
 def test_route_empty_batch(moe, cuda_device):
