@@ -588,6 +588,7 @@ bool ffn_shape_supported(int64_t H, int64_t I, moe_format_t fmt) {
 cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
                                const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows, void* ws,
                                cudaStream_t st) {
+  if (use_umma_path(T, E, k, ex.fmt)) return launch_grouped_ffn_umma(x, r, ex, T, H, I, E, k, y_rows, ws, st);
   switch (ex.fmt) {
     case MOE_FMT_W4G128:
       return launch_fmt<MOE_FMT_W4G128>(x, r, ex, bits, T, H, I, E, k, y_rows, ws, st);

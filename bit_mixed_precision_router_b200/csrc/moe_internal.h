@@ -30,6 +30,12 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const 
                                const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,
                                void* ws, cudaStream_t st);
 
+// Tensor-core (tcgen05) grouped GEMM path, used by launch_grouped_ffn when the
+// experts see enough rows on average (use_umma_path); W4 group-128 weights.
+bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt);
+cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
+                                    int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st);
+
 cudaError_t launch_combine(const uint16_t* y_rows, const moe_routing_t& r, const uint16_t* residual, int T,
                            int H, int k, uint16_t* out, cudaStream_t st);
 

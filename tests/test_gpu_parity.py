@@ -182,3 +182,31 @@ def test_grouped_ffn_and_combine(moe, cuda_device, fmt, T, H, I, E, k):
 
 def bf16_f64(b):
     return synth.bf16_bits_to_f32(b).astype(np.float64)
+
+
+# Batches with 32 or more rows per expert on average take the tensor-core GEMM
+# path (tcgen05, W4 group-128): 128-row tiles of weights and of routed rows.
+GEMM_CASES = [
+    # T, H, I, E, k, zipf
+    (512, 256, 128, 8, 2, False),     # ~128 rows per expert: one or two row tiles
+    (700, 512, 256, 16, 4, True),     # skewed: experts with several row tiles and empty ones
+    (300, 2048, 1024, 8, 2, False),   # OLMoE-like expert shape, 32 / 16 K-blocks
+    (129, 768, 384, 4, 1, False),     # ragged row tiles (MMA N not a multiple of 32), K = 768
+    (64, 256, 128, 1, 1, False),      # a single expert
+]
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", GEMM_CASES)
+def test_grouped_gemm_path(moe, cuda_device, T, H, I, E, k, zipf):
+    assert T * k >= 32 * E
+    L = make_layer(3000 + T + E, T, H, I, E, k, zipf=zipf)
+    ex_o = oracle_experts(FMT_W4G128, L.w13, L.w2)
+    ex_g = moe.quantize_experts(FMT_W4G128, dev_bf16(L.w13), dev_bf16(L.w2))
+    out, (logits, ids, w, offsets, sp, p2r) = _route_both(moe, L, k)
+    assert np.array_equal(out.sorted_pair.cpu().numpy(), sp)
+    y = moe.moe_grouped_ffn(dev_bf16(L.x), out, ex_g, I, E, k)
+    o = moe.moe_combine(y, out, T, k)
+    moe.moe_check_device_errors()
+    y_ref = grouped_ffn(L.x, offsets, sp, k, ex_o, None)
+    check_close(bf16_f64(host_bits(y)), y_ref, "y_rows (GEMM path)")
+    check_close(bf16_f64(host_bits(o)), combine(y_ref, w, p2r, None), "out (GEMM path)")
