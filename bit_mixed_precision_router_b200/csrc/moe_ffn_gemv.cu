@@ -490,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
 // ---------------------------------------------------------------- launch planning
 static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
-size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t /*E*/, int64_t k, moe_format_t /*fmt*/) {
+size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, moe_format_t fmt) {
+  if (use_umma_path(T, E, k, fmt)) return umma_workspace_bytes(T, H, I, k);
   return align256(size_t(T * k * I * 2));  // h
 }
 

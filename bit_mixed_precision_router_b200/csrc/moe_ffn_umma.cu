@@ -7,33 +7,41 @@
 // i.e. the same contraction as the weight-streaming GEMV, organised as a GEMM
 // when each expert sees enough rows for the weights to be worth reusing.
 //
-// Tile = 128 weight rows (the tensor-memory lanes, MMA M) x up to 128 rows of the
-// expert (MMA N) x the whole K.  For gate/up, the 128 weight rows are 64 gate rows
-// and the 64 matching up rows, arranged so that each warp quarter of the lanes
-// holds 16 gate rows and their 16 up rows: the SwiGLU product is formed in the
-// epilogue with one lane exchange.
-// Roles inside one persistent CTA (one per SM, 384 threads):
-//   warps 0-1   copy the B operand (token rows, bf16) with cp.async into a 6-stage
-//               ring of 128-byte-swizzled K-major tiles in shared memory;
-//   warp  2     allocates tensor memory and issues tcgen05.mma (kind::f16, bf16 in,
-//               fp32 accumulate) from one thread, A from tensor memory, B from
-//               shared memory; tcgen05.commit releases the stages;
-//   warps 4-7   dequantise the packed weights of their 32 rows each straight into
-//               tensor memory (tcgen05.st, 4 stages of 64 K-elements): the weight
-//               operand never passes through shared memory;
-//   warps 8-11  drain one of the two accumulators (tcgen05.ld) while the other is
+// Tile = 128 weight rows (the tensor-memory lanes, MMA M) x up to 192 routed rows
+// (MMA N) x the whole K.  For gate/up, the 128 weight rows are 64 gate rows and
+// the 64 matching up rows, arranged so that each warp quarter of the lanes holds
+// 16 gate rows and their 16 up rows: the SwiGLU product is formed in the epilogue
+// with one lane exchange.
+// Roles inside one persistent CTA (one per SM, 512 threads):
+//   warp  0     TMA producer: per 64-wide K block, the packed weight tile (4 KiB)
+//               into an 8-stage ring and the routed rows (bf16, 128-byte swizzled
+//               K-major, one 2-D box) into a 6-stage ring.  For gate/up the rows
+//               are the tokens gathered into routed order by k_gather_rows first
+//               (one bandwidth-bound pass; gathering 4 rows per TMA instruction
+//               inside the GEMM could not feed the tensor cores);
+//   warp  1     allocates tensor memory; one thread issues tcgen05.mma (kind::f16,
+//               bf16 in, fp32 accumulate), A from tensor memory, B from shared
+//               memory; tcgen05.commit releases the stages;
+//   warps 4-11  dequantise the weights from shared memory straight into tensor
+//               memory (tcgen05.st, 4 stages of 64 K): warp 4 + 4 s + q handles
+//               rows 32 q .. 32 q + 31 of the K blocks n with n % 2 == s, so two
+//               warps per sub-partition overlap each other's waits; the bf16
+//               weight operand never exists in shared memory;
+//   warps 12-15 drain one of the two accumulators (tcgen05.ld) while the other is
 //               being accumulated, apply SwiGLU, and store bf16 rows.
 // The work list (expert, row tile, weight tile) is built by every CTA from the
 // routing offsets and walked round-robin across CTAs.
 //
 // Dequantisation (W4 group-128): (u - 8) * s with u the stored nibble and s the
-// group's bf16 scale, formed as bf16 (128 + u) by bit operations, then
-// bf16 adds -136 exactly and multiplies by s with one rounding to bf16.  This is
-// the only rounding that differs from the fp32 dequantisation of the definition
-// (relative 2^-9 per weight, inside the FFN tolerance).
+// group's bf16 scale, formed as bf16 (128 + u) by byte permutes, then a bf16 add
+// of -136 (exact) and a bf16 multiply by s, rounded once.  That rounding is the
+// only difference from the fp32 dequantisation of the definition (relative 2^-9
+// per weight, inside the FFN tolerance).
 //
 // Every wait is bounded (mbar_wait): a wait that runs out sets the device error
 // word and the role stops; the CTA still frees its tensor memory.
+#include <cuda.h>  // CUtensorMap and its enums; the encoder is reached through the runtime
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -41,43 +49,44 @@ namespace moe {
 namespace {
 
 constexpr int kTM = 128;        // weight rows per tile (tensor-memory lanes)
-constexpr int kTN = 128;        // rows of the expert per tile (MMA N at most)
+constexpr int kTN = 192;        // routed rows per tile (MMA N at most)
 constexpr int kKB = 64;         // K elements per block: one 128-byte swizzle row of bf16
-constexpr int kBStages = 6;     // token-tile stages in shared memory
+constexpr int kBStages = 6;     // routed-row stages in shared memory
+constexpr int kWStages = 8;     // packed-weight stages in shared memory
 constexpr int kAStages = 4;     // dequantised weight stages in tensor memory
-constexpr int kLag = 3;         // cp.async groups kept in flight before a stage is published
-constexpr int kThreadsU = 384;
-constexpr int kTmemCols = 512;  // accumulators at columns 0 and 128, A stages at 256 + 32 a
-constexpr int kACol0 = 256;
+constexpr int kDeqSets = 2;     // dequantising warp sets, alternating K blocks
+constexpr int kThreadsU = 32 * (4 + 4 * kDeqSets + 4);
+constexpr int kTmemCols = 512;  // accumulators at columns 0 and 192, A stages at 384 + 32 a
+constexpr int kACol0 = 2 * kTN;
 constexpr int kBStageBytes = kTN * 128;
-constexpr int kPrefetch = 4;    // k-blocks of packed weights held in registers ahead
+constexpr int kWStageBytes = kTM * 32;  // 128 rows x 64 nibbles
+constexpr int kScaleAhead = 4;          // scale groups requested ahead by the dequantisers
 
-constexpr int kProdThreads = 64;
-constexpr int kMmaWarp = 2;
+constexpr int kProdWarp = 0;
+constexpr int kMmaWarp = 1;
 constexpr int kDeqWarp0 = 4;
-constexpr int kEpiWarp0 = 8;
+constexpr int kEpiWarp0 = kDeqWarp0 + 4 * kDeqSets;
 
 // shared memory plan (offsets from a 1024-byte aligned base)
 constexpr int kOffB = 0;
-constexpr int kOffPre = kOffB + kBStages * kBStageBytes;  // tile prefix over experts
+constexpr int kOffW = kOffB + kBStages * kBStageBytes;
+constexpr int kOffPre = kOffW + kWStages * kWStageBytes;  // tile prefix over experts
 constexpr int kOffBar = kOffPre + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
-constexpr int kNumBars = 2 * kBStages + 2 * kAStages + 4;
+constexpr int kNumBars = 2 * kBStages + 2 * kWStages + 2 * kAStages + 4;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffTmemSlot + 16;
-// + alignment slack; at least 120 KiB so that one CTA occupies an SM (and its
-// tensor memory) alone
-constexpr int kSmemBytes = (kSmemUsed + 1024) > 120 * 1024 ? (kSmemUsed + 1024) : 120 * 1024;
+constexpr int kSmemBytes = kSmemUsed + 1024;  // + alignment slack; > half an SM: one CTA per SM
+static_assert(kSmemBytes > 114 * 1024 && kSmemBytes <= 227 * 1024, "shared-memory plan");
+static_assert(kACol0 + kAStages * 32 <= kTmemCols, "tensor-memory plan");
 
 constexpr int kGateUp = 0, kDown = 1;
 
 struct UmmaArgs {
-  const uint16_t* act;       // gate/up: x [T][K]; down: h [P][K]
   int K, I, E, k;
   int wtiles;                // weight tiles per expert
   int n_rows;                // rows of one expert's weight matrix (2I or H)
   const int32_t* offsets;    // [E+1]
   const int32_t* sorted_pair;
-  const uint32_t* w;         // packed W4 [E][n_rows][K/8]
   const uint16_t* s;         // bf16 scales [E][n_rows][K/128]
   uint16_t* out;             // gate/up: h [P][I]; down: y [P][H]
   int out_ld;
@@ -141,17 +150,21 @@ MOE_DEVICE void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "memory");
 }
 
-MOE_DEVICE void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-MOE_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-MOE_DEVICE void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-MOE_DEVICE void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 MOE_DEVICE void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+// 2-D tiled tensor load (box of the map) at element coordinates (c0 inner, c1 outer).
+MOE_DEVICE void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+MOE_DEVICE uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
 }
 
 // mbar_wait taken by a whole warp: the result is the same in every lane, so the
@@ -178,9 +191,8 @@ MOE_DEVICE uint32_t idesc_bf16(int n) {
 }
 
 // ---------------------------------------------------------------- W4 dequant
-// Two nibbles a (low half) and b (high half) as bf16x2 (128 + a, 128 + b).
-// w holds elements 8i..8i+7 of one row (element j at bits 4j); the result pairs
-// (0,1), (2,3), (4,5), (6,7) in p[0..3].
+// w holds elements 8i..8i+7 of one row (element j at bits 4j); p[0..3] receive
+// the pairs (0,1), (2,3), (4,5), (6,7) as bf16x2 (128 + u_lo, 128 + u_hi).
 MOE_DEVICE void w4_word_pairs(uint32_t w, uint32_t (&p)[4]) {
   const uint32_t lo = w & 0x0F0F0F0Fu;         // n0 n2 n4 n6
   const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // n1 n3 n5 n7
@@ -192,7 +204,6 @@ MOE_DEVICE void w4_word_pairs(uint32_t w, uint32_t (&p)[4]) {
   p[2] = __byte_perm(u23, k43, 0x4140);
   p[3] = __byte_perm(u23, k43, 0x4342);
 }
-
 MOE_DEVICE uint32_t bf16x2_add(uint32_t a, uint32_t b) {
   __nv_bfloat162 r = __hadd2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
@@ -225,7 +236,8 @@ MOE_DEVICE Tile tile_of(int item, const int* pre, int E, int wtiles, const int32
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreadsU, 1) k_ffn_umma(UmmaArgs a) {
+__global__ void __launch_bounds__(kThreadsU, 1)
+    k_ffn_umma(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w, UmmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -233,8 +245,10 @@ __global__ void __launch_bounds__(kThreadsU, 1) k_ffn_umma(UmmaArgs a) {
   int* pre = reinterpret_cast<int*>(smem + kOffPre);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* fullB = bars;
-  uint64_t* emptyB = bars + kBStages;
-  uint64_t* fullA = bars + 2 * kBStages;
+  uint64_t* emptyB = fullB + kBStages;
+  uint64_t* fullW = emptyB + kBStages;
+  uint64_t* emptyW = fullW + kWStages;
+  uint64_t* fullA = emptyW + kWStages;
   uint64_t* emptyA = fullA + kAStages;
   uint64_t* accFull = emptyA + kAStages;
   uint64_t* accEmpty = accFull + 2;
@@ -243,7 +257,7 @@ __global__ void __launch_bounds__(kThreadsU, 1) k_ffn_umma(UmmaArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E;
 
-  // ---- tiles per expert and their prefix (warp 0), barriers (thread 32), tensor memory (warp 2)
+  // ---- tiles per expert and their prefix (warp 0), barriers (warp 2), tensor memory (warp 1)
   if (warp == 0) {
     const int per = (E + 31) / 32;
     const int b = min(E, lane * per), en = min(E, b + per);
@@ -261,13 +275,17 @@ __global__ void __launch_bounds__(kThreadsU, 1) k_ffn_umma(UmmaArgs a) {
       run += (a.offsets[e + 1] - a.offsets[e] + kTN - 1) / kTN;
     }
     if (lane == 31) pre[E] = inc;
-  } else if (tid == 32) {
+  } else if (tid == 64) {
     for (int i = 0; i < kBStages; ++i) {
-      mbar_init(&fullB[i], kProdThreads);
+      mbar_init(&fullB[i], 1);
       mbar_init(&emptyB[i], 1);
     }
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&fullW[i], 1);
+      mbar_init(&emptyW[i], 4);
+    }
     for (int i = 0; i < kAStages; ++i) {
-      mbar_init(&fullA[i], 4);
+      mbar_init(&fullA[i], 4);  // the four warps of the set that wrote the stage
       mbar_init(&emptyA[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -286,159 +304,151 @@ __global__ void __launch_bounds__(kThreadsU, 1) k_ffn_umma(UmmaArgs a) {
   const int n_items = pre[E] * a.wtiles;
   const int KB = a.K / kKB;
 
-  if (tid < kProdThreads) {
-    // ------------------------------------------------ B producer (token rows)
-    // thread: chunk c = tid % 8 of rows rr = tid / 8 + 8 i (i < 16); the chunk lands
-    // at c ^ (row % 8) = c ^ (tid / 8) inside its 128-byte row
-    const int c = tid & 7, rsub = tid >> 3;
-    const uint32_t dst_off = uint32_t(rsub * 128 + ((c ^ rsub) << 4));
-    int n = 0;  // stages issued
+  if (warp == kProdWarp) {
+    // ------------------------------------------------ TMA producer
+    int n = 0;  // k-blocks issued
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
-      // gate/up: the token of each row; down: rows r0 + rr of h, 8 rows apart
-      const uint16_t* src[MODE == kGateUp ? 16 : 1];
+      int wr0, wr1;  // weight box rows
       if (MODE == kGateUp) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int rr = rsub + 8 * i;
-          const int r = tl.r0 + (rr < tl.nrows ? rr : 0);
-          src[i] = a.act + size_t(a.sorted_pair[r] / a.k) * a.K + c * 8;
-        }
+        wr0 = tl.e * a.n_rows + tl.wt * 64;
+        wr1 = wr0 + a.I;
       } else {
-        src[0] = a.act + size_t(tl.r0 + rsub) * a.K + c * 8;
+        wr0 = tl.e * a.n_rows + tl.wt * kTM;
+        wr1 = 0;
       }
       for (int kb = 0; kb < KB; ++kb, ++n) {
-        const int st = n % kBStages;
-        if (!mbar_wait(&emptyB[st], ((n / kBStages) & 1) ^ 1, a.err)) {
+        const int sw = n % kWStages, sb = n % kBStages;
+        if (!warp_wait(&emptyW[sw], ((n / kWStages) & 1) ^ 1, a.err)) {
           ok = false;
           break;
         }
-        const uint32_t dst = sbase + kOffB + st * kBStageBytes + dst_off;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (rsub + 8 * i < tl.nrows)
-            cp_async16(dst + i * 1024, (MODE == kGateUp ? src[i] : src[0] + size_t(8 * i) * a.K) + kb * kKB);
-        cp_async_commit();
-        if (n >= kLag) {
-          cp_async_wait<kLag>();
-          fence_async_smem();
-          mbar_arrive(&fullB[(n - kLag) % kBStages]);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&fullW[sw], uint32_t(kWStageBytes));
+          const uint32_t wdst = sbase + kOffW + sw * kWStageBytes;
+          if (MODE == kGateUp) {
+            tma_load_2d(wdst, &tm_w, kb * 32, wr0, &fullW[sw]);
+            tma_load_2d(wdst + kWStageBytes / 2, &tm_w, kb * 32, wr1, &fullW[sw]);
+          } else {
+            tma_load_2d(wdst, &tm_w, kb * 32, wr0, &fullW[sw]);
+          }
+        }
+        if (!warp_wait(&emptyB[sb], ((n / kBStages) & 1) ^ 1, a.err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bdst = sbase + kOffB + sb * kBStageBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&fullB[sb], uint32_t(kBStageBytes));
+          tma_load_2d(bdst, &tm_b, kb * kKB, tl.r0, &fullB[sb]);
         }
       }
     }
-    // publish the stages still in flight
-    cp_async_wait<0>();
-    fence_async_smem();
-    for (int m = (n > kLag ? n - kLag : 0); m < n; ++m) mbar_arrive(&fullB[m % kBStages]);
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------ MMA issuer
-    int nb = 0, na = 0, it = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
-      const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
-      const int ab = it & 1;
-      if (!warp_wait(&accEmpty[ab], ((it >> 1) & 1) ^ 1, a.err)) break;
-      tc_fence_after();
-      const int nmma = (tl.nrows + 15) & ~15;
-      const uint32_t idesc = idesc_bf16(nmma);
-      const uint32_t d_tmem = tmem + uint32_t(ab * kTN);
-      for (int kb = 0; kb < KB; ++kb, ++nb, ++na) {
-        const int sb = nb % kBStages, sa = na % kAStages;
-        if (!warp_wait(&fullB[sb], (nb / kBStages) & 1, a.err) || !warp_wait(&fullA[sa], (na / kAStages) & 1, a.err)) {
-          ok = false;
-          break;
-        }
+    // ------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      int n = 0, it = 0;
+      bool ok = true;
+      const uint64_t bdesc0 = sw128_desc(sbase + kOffB);
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
+        const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
+        const int ab = it & 1;
+        if (!mbar_wait(&accEmpty[ab], ((it >> 1) & 1) ^ 1, a.err)) break;
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t b_addr = sbase + kOffB + sb * kBStageBytes;
+        const uint32_t idesc = idesc_bf16((tl.nrows + 15) & ~15);
+        const uint32_t d_tmem = tmem + uint32_t(ab * kTN);
+        for (int kb = 0; kb < KB; ++kb, ++n) {
+          const int sb = n % kBStages, sa = n % kAStages;
+          if (!mbar_wait(&fullA[sa], (n / kAStages) & 1, a.err) || !mbar_wait(&fullB[sb], (n / kBStages) & 1, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = bdesc0 + uint64_t((sb * kBStageBytes) >> 4);
           const uint32_t a_tmem = tmem + uint32_t(kACol0 + sa * 32);
 #pragma unroll
           for (int kk = 0; kk < kKB / 16; ++kk)
-            tc_mma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b_addr + kk * 32), idesc, (kb | kk) != 0);
+            tc_mma_ts(d_tmem, a_tmem + kk * 8, bdesc + uint64_t(2 * kk), idesc, (kb | kk) != 0);
           tc_commit(&emptyB[sb]);
           tc_commit(&emptyA[sa]);
         }
-        __syncwarp();
+        if (ok) tc_commit(&accFull[ab]);
       }
-      if (ok && lane == 0) tc_commit(&accFull[ab]);
-      __syncwarp();
+      // the last accumulation must be complete before the tensor memory is freed
+      if (it > 0 && ok) mbar_wait(&accFull[(it - 1) & 1], ((it - 1) >> 1) & 1, a.err);
     }
-    // the last accumulation must be complete before the tensor memory is freed
-    if (it > 0 && ok) mbar_wait(&accFull[(it - 1) & 1], (((it - 1) >> 1) & 1), a.err);
-  } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + 4) {
+    __syncwarp();
+  } else if (warp >= kDeqWarp0 && warp < kEpiWarp0) {
     // ------------------------------------------------ dequantise W into tensor memory
-    // This CTA's k-blocks form one stream (its items in order, K blocks each); the
-    // packed words and scale of block g + kPrefetch are requested while block g is
-    // converted, across item boundaries too.
-    const int quarter = warp - kDeqWarp0;
+    const int quarter = (warp - kDeqWarp0) & 3, set = (warp - kDeqWarp0) >> 2;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
-    const int KW = a.K / 8, KG = a.K / 128;
+    const int KG = a.K / 128;
+    // row of this lane inside the weight box(es); for gate/up, lanes 0-15 of each
+    // quarter hold gate rows and lanes 16-31 the up rows of the same 16 columns
+    const int srow = (MODE == kGateUp) ? ((lane < 16) ? quarter * 16 + lane : 64 + quarter * 16 + (lane - 16))
+                                       : quarter * 32 + lane;
     const int my_items = blockIdx.x < n_items ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
     const int total = my_items * KB;
-    // weight row of this lane in tile column wt: for gate/up, lanes 0-15 of each
-    // quarter hold gate rows and lanes 16-31 the up rows of the same 16 columns
-    auto row_of = [&](int item) -> size_t {
-      const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
-      int n;
-      if (MODE == kGateUp) {
-        const int i = tl.wt * 64 + quarter * 16 + (lane & 15);
-        n = (lane < 16) ? i : a.I + i;
-      } else {
-        n = tl.wt * kTM + quarter * 32 + lane;
+    // scales: one bf16 per 128 K (every other block), requested kScaleAhead groups ahead
+    int s_li = -1;
+    const uint16_t* s_row = nullptr;
+    auto scale_at = [&](int g2) -> uint32_t {  // g2 = flat index of a 128-wide group
+      const int li = (2 * g2) / KB, grp = g2 - li * (KB / 2);
+      if (li != s_li) {
+        s_li = li;
+        const Tile tl = tile_of(int(blockIdx.x) + li * int(gridDim.x), pre, E, a.wtiles, a.offsets);
+        int n;
+        if (MODE == kGateUp) n = (srow < 64) ? tl.wt * 64 + srow : a.I + tl.wt * 64 + (srow - 64);
+        else n = tl.wt * kTM + srow;
+        s_row = a.s + (size_t(tl.e) * a.n_rows + n) * KG;
       }
-      return size_t(tl.e) * a.n_rows + n;
+      return s_row[grp];
     };
-    int p_idx = -1;  // local item index whose row pointers are cached
-    const uint4* p_wp = nullptr;
-    const uint16_t* p_sp = nullptr;
-    auto fetch = [&](int g, uint4& w0, uint4& w1, uint16_t& sv) {
-      const int li = g / KB, kb = g - li * KB;
-      if (li != p_idx) {
-        p_idx = li;
-        const size_t row = row_of(int(blockIdx.x) + li * int(gridDim.x));
-        p_wp = reinterpret_cast<const uint4*>(a.w + row * KW);
-        p_sp = a.s + row * KG;
-      }
-      w0 = ldg_nc_v4(p_wp + 2 * kb);
-      w1 = ldg_nc_v4(p_wp + 2 * kb + 1);
-      sv = p_sp[kb >> 1];
-    };
-    uint4 ring0[kPrefetch], ring1[kPrefetch];
-    uint16_t rings[kPrefetch];
+    uint32_t sring[kScaleAhead];
+    const int total_g = total / 2;
 #pragma unroll
-    for (int q = 0; q < kPrefetch; ++q)
-      if (q < total) fetch(q, ring0[q], ring1[q], rings[q]);
+    for (int q = 0; q < kScaleAhead; ++q) sring[q] = (q < total_g) ? scale_at(q) : 0u;
     bool ok = true;
-    for (int g0 = 0; g0 < total && ok; g0 += kPrefetch) {
+    for (int g0 = 0; g0 < total_g && ok; g0 += kScaleAhead) {
 #pragma unroll
-      for (int q = 0; q < kPrefetch; ++q) {
-        const int g = g0 + q;
-        if (g >= total) break;
-        const uint4 w0 = ring0[q], w1 = ring1[q];
-        const uint32_t sv = rings[q];
-        if (g + kPrefetch < total) fetch(g + kPrefetch, ring0[q], ring1[q], rings[q]);
+      for (int q = 0; q < kScaleAhead; ++q) {
+        const int g2 = g0 + q;
+        if (g2 >= total_g) break;
+        const uint32_t sv = sring[q];
+        if (g2 + kScaleAhead < total_g) sring[q] = scale_at(g2 + kScaleAhead);
         const uint32_t s2 = sv | (sv << 16);
-        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint32_t v[32];
+        {
+          const int n = 2 * g2 + set;
+          const int sw = n % kWStages, sa = n % kAStages;
+          if (!warp_wait(&fullW[sw], (n / kWStages) & 1, a.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t wrow = sbase + kOffW + sw * kWStageBytes + srow * 32;
+          const uint4 w0 = lds128(wrow), w1 = lds128(wrow + 16);
+          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          uint32_t v[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint32_t p[4];
-          w4_word_pairs(words[i], p);
+          for (int i = 0; i < 8; ++i) {
+            uint32_t p[4];
+            w4_word_pairs(words[i], p);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) v[4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
+            for (int j = 0; j < 4; ++j) v[4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&emptyW[sw]);
+          if (!warp_wait(&emptyA[sa], ((n / kAStages) & 1) ^ 1, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tmem_st32(tmem + lane_base + uint32_t(kACol0 + sa * 32), v);
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&fullA[sa]);
         }
-        const int sa = g % kAStages;
-        if (!warp_wait(&emptyA[sa], ((g / kAStages) & 1) ^ 1, a.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st32(tmem + lane_base + uint32_t(kACol0 + sa * 32), v);
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&fullA[sa]);
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -486,6 +496,61 @@ __global__ void __launch_bounds__(kThreadsU, 1) k_ffn_umma(UmmaArgs a) {
   }
 }
 
+// xs[r] = x[sorted_pair[r] / k]: the token rows in routed order; one warp per row,
+// 16 bytes per lane per step, four steps in flight.
+__global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_pair,
+                                                     int P, int k, int row16, uint4* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = int(gridDim.x) * (blockDim.x >> 5);
+  for (int r = int(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += nwarps) {
+    const uint4* src = x + int64_t(__ldg(sorted_pair + r) / k) * row16;
+    uint4* dst = xs + int64_t(r) * row16;
+    for (int c0 = 0; c0 < row16; c0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u + lane;
+        if (c < row16) v[u] = __ldg(src + c);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u + lane;
+        if (c < row16) dst[c] = v[u];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows][cols] array with `row_bytes` between rows.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+                 uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int cached[128] = {};
   int dev = 0;
@@ -499,34 +564,42 @@ int sm_count() {
 }
 
 template <int MODE>
-cudaError_t launch_umma_one(const UmmaArgs& a, cudaStream_t st) {
+cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const UmmaArgs& a, cudaStream_t st) {
   static bool raised[128] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!raised[dev]) {
-    const cudaError_t err = cudaFuncSetAttribute(k_ffn_umma<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const cudaError_t err =
+        cudaFuncSetAttribute(k_ffn_umma<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
     raised[dev] = true;
   }
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  k_ffn_umma<MODE><<<nsm, kThreadsU, kSmemBytes, st>>>(a);
+  k_ffn_umma<MODE><<<nsm, kThreadsU, kSmemBytes, st>>>(tb, tw, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 // At 32 or more rows per expert on average, the tensor-core GEMM (weights
-// dequantised once per 128 rows) beats streaming the weights once per 16 rows.
+// dequantised once per 192 rows) beats streaming the weights once per 16 rows.
 bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt) {
   return fmt == MOE_FMT_W4G128 && T * k >= 32 * E;
 }
 
+static size_t align256u(size_t b) { return (b + 255) / 256 * 256; }
+size_t umma_h_bytes(int64_t T, int64_t I, int64_t k) { return align256u(size_t(T * k * I * 2)); }
+// h [P][I] bf16, then the routed token rows [P][H] bf16
+size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k) {
+  return umma_h_bytes(T, I, k) + align256u(size_t(T * k * H * 2));
+}
+
 cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
                                     int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st) {
-  (void)T;
   if (ex.fmt != MOE_FMT_W4G128) return cudaErrorInvalidValue;
+  const int P = T * k;
   UmmaArgs a{};
   a.E = E;
   a.k = k;
@@ -535,27 +608,42 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
   a.sorted_pair = r.sorted_pair;
   a.err = device_error_word();
   if (!a.err) return cudaErrorInvalidDevice;
-  // gate/up: weight tiles of 64 gate + 64 up rows
-  a.act = x;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  // the token rows in routed order, after h in the workspace
+  uint16_t* xs = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(hbuf) + umma_h_bytes(T, I, k));
+  k_gather_rows<<<4 * nsm, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), r.sorted_pair, P, k, H / 8,
+                                         reinterpret_cast<uint4*>(xs));
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  CUtensorMap tb, tw;
+  // gate/up: routed token rows in one box per stage; weight boxes of 64 gate and 64 up rows
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs, uint64_t(H), uint64_t(P), uint64_t(H) * 2, kKB, kTN,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w13, uint64_t(H) / 2, uint64_t(E) * 2 * I,
+                   uint64_t(H) / 2, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   a.K = H;
   a.n_rows = 2 * I;
   a.wtiles = I / 64;
-  a.w = static_cast<const uint32_t*>(ex.w13);
   a.s = static_cast<const uint16_t*>(ex.w13_scale);
   a.out = static_cast<uint16_t*>(hbuf);
   a.out_ld = I;
-  cudaError_t err = launch_umma_one<kGateUp>(a, st);
+  err = launch_umma_one<kGateUp>(tb, tw, a, st);
   if (err != cudaSuccess) return err;
-  // down
-  a.act = static_cast<const uint16_t*>(hbuf);
+  // down: h rows in one box per stage; weight boxes of 128 rows
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hbuf, uint64_t(I), uint64_t(P), uint64_t(I) * 2, kKB,
+                   kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 32,
+                   kTM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   a.K = I;
   a.n_rows = H;
   a.wtiles = H / kTM;
-  a.w = static_cast<const uint32_t*>(ex.w2);
   a.s = static_cast<const uint16_t*>(ex.w2_scale);
   a.out = y_rows;
   a.out_ld = H;
-  return launch_umma_one<kDown>(a, st);
+  return launch_umma_one<kDown>(tb, tw, a, st);
 }
 
 }  // namespace moe

@@ -33,6 +33,8 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const 
 // Tensor-core (tcgen05) grouped GEMM path, used by launch_grouped_ffn when the
 // experts see enough rows on average (use_umma_path); W4 group-128 weights.
 bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt);
+size_t umma_h_bytes(int64_t T, int64_t I, int64_t k);
+size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
 cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
                                     int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st);
 
