@@ -11,6 +11,11 @@ as one CUDA graph.  `value` = tokens per second through the 16-layer stack
 (a token counts once per step), whole job over all ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl reference]
+                    [--workload decode|prefill-h2048-e128|prefill-h7168-e256]
+
+The prefill workloads (not the default) time one MoE FFN layer on a large batch
+of fresh tokens per step -- the tensor-core grouped GEMM path -- and report its
+roofline against the measured bf16 tensor peak.
 
 Under torchrun each rank runs its own replica on its own seeded batches (the
 layer shards by token, no data-path collective): weak scaling, time = max over
@@ -38,11 +43,22 @@ W4_EXPERT_BYTES = (2 * I * H + H * I) // 2 + (2 * I * (H // 128) + H * (I // 128
 W13_EXPERT_BYTES = 2 * I * H // 2 + 2 * I * (H // 128) * 2
 W2_EXPERT_BYTES = H * I // 2 + H * (I // 128) * 2
 
+# Prefill-sized single layers (W4A16 g128 experts): shapes, routing and seeds.
+PREFILL = {
+    "prefill-h2048-e128": dict(T=2048, H=2048, I=768, E=128, k=8, router="normal", zipf=True, seed=0x5EED0003,
+                               desc="one MoE FFN layer, H2048 I768 E128 top-8, W4A16 g128 experts, bf16 router "
+                                    "with a Zipf(1.1) rank bias, 2048 fresh tokens per step"),
+    "prefill-h7168-e256": dict(T=4096, H=7168, I=2048, E=256, k=8, router="uniform", zipf=False, seed=0x5EED0005,
+                               desc="one MoE FFN layer, H7168 I2048 E256 top-8, W4A16 g128 experts, "
+                                    "U(-0.02, 0.02) bf16 router, 4096 fresh tokens per step"),
+}
+
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--workload", choices=["decode"] + sorted(PREFILL), default="decode")
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 512 decode, 20 prefill)")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--batch", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -50,7 +66,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers in the stack (16 is the benchmark workload; fewer only for profiling)")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = 512 if args.workload == "decode" else 20
+    return args
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -361,6 +380,208 @@ def run_gpu(args, rank, world, local):
     return result
 
 
+# ---------------------------------------------------------------- prefill workloads
+class PrefillLayer:
+    """One W4A16 MoE FFN layer made on the device (seeded generator, quantised in
+    chunks of experts) with every buffer a prefill step needs."""
+
+    def __init__(self, moe, torch, device, cfg, chunk=16):
+        import synth
+        self.moe, self.cfg = moe, cfg
+        T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
+        seed = cfg["seed"]
+        i32, bf = dict(dtype=torch.int32, device=device), dict(dtype=torch.bfloat16, device=device)
+        w13q, w13s = torch.empty((Ee, 2 * Ii, Hh // 8), **i32), torch.empty((Ee, 2 * Ii, Hh // 128), **bf)
+        w2q, w2s = torch.empty((Ee, Hh, Ii // 8), **i32), torch.empty((Ee, Hh, Ii // 128), **bf)
+        tmp = torch.empty((chunk * 2 * Ii * Hh,), **bf)
+        for (n, kk, tag, q, sc) in ((2 * Ii, Hh, synth.SEED_W13, w13q, w13s), (Hh, Ii, synth.SEED_W2, w2q, w2s)):
+            for e0 in range(0, Ee, chunk):
+                ne = min(chunk, Ee - e0)
+                t = tmp[:ne * n * kk].view(ne, n, kk)
+                moe.moe_synth_normal_bf16(t, seed + tag, 0.02, start=e0 * n * kk)
+                moe.moe_quantize_w4g128(t, q[e0:e0 + ne], sc[e0:e0 + ne])
+        del tmp
+        self.experts = moe.Experts(moe.FMT_W4G128, w13q, w13s, w2q, w2s)
+        self.wr = torch.empty((Ee, Hh), **bf)
+        if cfg["router"] == "uniform":
+            moe.moe_synth_uniform_bf16(self.wr, seed + synth.SEED_WR, -0.02, 0.02)
+        else:
+            moe.moe_synth_normal_bf16(self.wr, seed + synth.SEED_WR, 0.02)
+        self.bias = torch.from_numpy(synth.zipf_rank_bias(seed + synth.SEED_BIAS, Ee)).to(device) \
+            if cfg["zipf"] else None
+        self.routing = moe.Routing.empty(T, Ee, k, device)
+        self.route_ws = moe.moe_route_workspace(T, Ee, k, device)
+        self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(T, Hh, Ii, Ee, k, moe.FMT_W4G128), 16),
+                                  dtype=torch.uint8, device=device)
+        self.y_rows = torch.empty((T * k, Hh), **bf)
+        self.x = torch.empty((T, Hh), **bf)
+        self.out = torch.empty((T, Hh), **bf)
+        self.ffn_events = None
+
+    def step(self):
+        moe, c = self.moe, self.cfg
+        moe.moe_route_topk(self.x, self.wr, self.bias, c["k"], out=self.routing, workspace=self.route_ws)
+        if self.ffn_events is not None:
+            self.ffn_events[0].record()
+        moe.moe_grouped_ffn(self.x, self.routing, self.experts, c["I"], c["E"], c["k"], y_rows=self.y_rows,
+                            workspace=self.ffn_ws)
+        if self.ffn_events is not None:
+            self.ffn_events[1].record()
+        moe.moe_combine(self.y_rows, self.routing, c["T"], c["k"], residual=self.x, out=self.out)
+
+    kernels_per_step = 7  # router logits, top-k, permutation, row gather, gate/up GEMM, down GEMM, combine
+
+
+def run_prefill(args, rank, world, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import bit_mixed_precision_router_b200 as moe
+    moe.load()
+    import synth
+    cfg = PREFILL[args.workload]
+    T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
+    K, W = args.steps, max(args.warmup, 3)
+    layer = PrefillLayer(moe, torch, device, cfg)
+    inputs = torch.empty((W + K, T, Hh), dtype=torch.bfloat16, device=device)
+    moe.moe_synth_normal_bf16(inputs, rank_seed(cfg["seed"], rank) + synth.SEED_X, 1.0)
+    torch.cuda.synchronize()
+    layer.x.copy_(inputs[0])
+    layer.step()  # eager first call: device symbols and kernel attributes before capture
+    torch.cuda.synchronize()
+    moe.moe_check_device_errors()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device)
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            layer.step()
+    torch.cuda.current_stream().wait_stream(cap)
+    for s in range(W):
+        layer.x.copy_(inputs[s])
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for s in range(W, W + K):
+        layer.x.copy_(inputs[s])
+        graph.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    moe.moe_check_device_errors()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    tokens = T * K * world
+    value = tokens / (ms / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        host_in = inputs[W:W + K].cpu().pin_memory()
+        host_out = torch.empty((K, T, Hh), dtype=torch.bfloat16).pin_memory()
+        barrier(world)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for s in range(K):
+            layer.x.copy_(host_in[s], non_blocking=True)
+            graph.replay()
+            host_out[s].copy_(layer.out, non_blocking=True)
+        t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * Hh * 2,
+               "d2h_bytes_per_step": T * Hh * 2}
+
+    # roofline of the dominant op: the grouped GEMM (row gather + gate/up + down launches
+    # of moe_grouped_ffn), CUDA events recorded on its stream inside a graph
+    layer.ffn_events = (torch.cuda.Event(enable_timing=True, external=True),
+                        torch.cuda.Event(enable_timing=True, external=True))
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g2, stream=cap):
+            layer.step()
+    torch.cuda.current_stream().wait_stream(cap)
+    ffn_ms = []
+    for s in range(W, W + min(K, 10)):
+        layer.x.copy_(inputs[s])
+        g2.replay()
+        torch.cuda.synchronize()
+        ffn_ms.append(layer.ffn_events[0].elapsed_time(layer.ffn_events[1]))
+    layer.ffn_events = None
+    hbm, bf16_peak, peak_kind = measured_peaks()
+    flops = 2.0 * T * k * 3 * Hh * Ii
+    avg_s = statistics.mean(ffn_ms) / 1e3
+    achieved = flops / avg_s / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / bf16_peak, 4), "peak_kind": peak_kind + " bf16 burst", "traffic": None,
+                "kernel": "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
+                "algorithmic_flops_per_call": flops, "avg_call_us": round(avg_s * 1e6, 1)}
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, "
+                                                          "N(0,0.02) bf16 weights quantised to W4A16 g128)",
+            "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,
+                       "top_k": k, "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "no flush: each step reads %.2f GB of expert weights, > 126 MB L2"
+                             % (Ee * (3 * Hh * Ii // 2 + 3 * Hh * Ii // 64) / 1e9)},
+            "gpu_launches": PrefillLayer.kernels_per_step * K,
+            "clocks": clk, "roofline": roofline, "e2e": e2e,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        del graph, g2
+        dist.destroy_process_group()
+    return result
+
+
+def oracle_prefill_sample(cfg, tokens: int, seed: int):
+    """Times the CPU oracle on `tokens` tokens of one prefill layer (routing, the routed
+    experts' dequantisation and SwiGLU, combine); the experts' weights are generated and
+    quantised untimed.  Returns (tokens/s, seconds timed, threads)."""
+    import numpy as np
+
+    import synth
+    from oracle.ffn import FMT_W4G128, Experts, moe_layer
+    from oracle.quant import quantize_w4g128
+    from oracle.routing import router_logits, topk_softmax
+    T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
+    x = synth.normal_bf16(seed + synth.SEED_X, tokens * Hh, 1.0).reshape(tokens, Hh)
+    if cfg["router"] == "uniform":
+        wr = synth.uniform_bf16(cfg["seed"] + synth.SEED_WR, Ee * Hh, -0.02, 0.02).reshape(Ee, Hh)
+    else:
+        wr = synth.normal_bf16(cfg["seed"] + synth.SEED_WR, Ee * Hh, 0.02).reshape(Ee, Hh)
+    bias = synth.zipf_rank_bias(cfg["seed"] + synth.SEED_BIAS, Ee) if cfg["zipf"] else None
+    ids, _ = topk_softmax(router_logits(x, wr, bias), k)
+    w13q = np.zeros((Ee, 2 * Ii, Hh // 8), np.uint32)
+    w13s = np.zeros((Ee, 2 * Ii, Hh // 128), np.uint16)
+    w2q = np.zeros((Ee, Hh, Ii // 8), np.uint32)
+    w2s = np.zeros((Ee, Hh, Ii // 128), np.uint16)
+    for e in sorted(set(ids.reshape(-1).tolist())):
+        a = quantize_w4g128(synth.normal_rows_bf16(cfg["seed"] + synth.SEED_W13, (2 * Ii, Hh), 0.02, e, 1))
+        b = quantize_w4g128(synth.normal_rows_bf16(cfg["seed"] + synth.SEED_W2, (Hh, Ii), 0.02, e, 1))
+        w13q[e], w13s[e], w2q[e], w2s[e] = a[0][0], a[1][0], b[0][0], b[1][0]
+    ex = Experts(FMT_W4G128, w13q, w13s, w2q, w2s)
+    t0 = time.perf_counter()
+    moe_layer(x, wr, bias, ex, k, residual_bits=x)
+    secs = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    return tokens / secs, secs, threads
+
+
 # ---------------------------------------------------------------- the oracle (CPU) arm
 def oracle_sample(batch: int, layers_timed: int, seed: int):
     """Times the CPU oracle on a bounded sample of the decode stack: `layers_timed`
@@ -400,6 +621,18 @@ def oracle_sample(batch: int, layers_timed: int, seed: int):
     return batch / per_step, timed, threads
 
 
+def prefill_sample_tokens(cfg) -> int:
+    return 2 if cfg["H"] > 4096 else 32  # bounded: a few to about 30 s of oracle work
+
+
+def cpu_baseline_prefill(cfg, seed: int):
+    n = prefill_sample_tokens(cfg)
+    v, secs, thr = oracle_prefill_sample(cfg, n, seed)
+    return {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{n} tokens through the layer ({secs:.1f} s of CPU work: routing, dequantisation of "
+                      f"their experts, SwiGLU, combine); weights generated and quantised untimed"}
+
+
 def cpu_baseline(batch: int, seed: int):
     layers_timed = 2
     v, secs, thr = oracle_sample(batch, layers_timed, seed)
@@ -412,6 +645,18 @@ def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on this workload's config."""
     if rank != 0:
         return None
+    if args.workload != "decode":
+        cfg = PREFILL[args.workload]
+        n = prefill_sample_tokens(cfg)
+        v, secs, thr = oracle_prefill_sample(cfg, n, cfg["seed"])
+        return {"metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(cfg["T"] / v * 1e3, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": cfg["desc"], "tokens": cfg["T"]},
+                "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                                 "sample": f"{n} tokens through the layer ({secs:.1f} s), scaled per token"},
+                "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     B = args.batch
     K, W = args.steps, args.warmup
     # each step: a bounded sample (2 layers of the stack), W + K of them kept short
@@ -440,6 +685,13 @@ def main(argv=None):
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    if args.workload != "decode":
+        res = run_prefill(args, rank, world, local)
+        if rank == 0 and res is not None and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline_prefill(PREFILL[args.workload], PREFILL[args.workload]["seed"])
+        if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
         return 0
     res = run_gpu(args, rank, world, local)

@@ -8,11 +8,12 @@
 // One CTA = one routed expert x 8 warps, each warp owning whole units.  The expert's
 // activations for a chunk of up to `nx` tokens are staged once per CTA in shared memory,
 // already paired the way the dequantised weights pair them and with their per-group sums.
-// Each warp then streams its own units group by group (16 rows x 128 K-elements per step)
-// through a private ring of shared-memory slots with 16-byte cp.async copies kept kDepth
-// steps ahead (commit/wait groups, no cross-warp handshake), and per step: shared loads,
-// nibble / bit / FP4 -> bf16 (fp16) in registers, mma.sync m16n8k16 with the tokens on N.
-// Expert weights are read from HBM once per token chunk.
+// Each warp then streams its own units group by group (16 rows x 128 K-elements per group)
+// through a private ring of shared-memory slots with 16-byte cp.async copies kept several
+// groups ahead (commit/wait groups, no cross-warp handshake), and per group: shared loads,
+// nibble / bit / FP4 -> fp16 or bf16 in registers, mma.sync m16n8k16 with the tokens on N.
+// W4 takes two groups per wait and converts nibbles to fp16 against activations staged
+// in fp16 (see w4h_group).  Expert weights are read from HBM once per token chunk.
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
@@ -25,7 +26,8 @@ enum { kGateUp = 0, kDown = 1 };
 constexpr int kRows = 16;     // weight rows per unit
 constexpr int kWarps = 8;     // warps per CTA, each owning whole units
 constexpr int kThreads = 32 * kWarps;
-constexpr int kDepth = 6;     // group steps in flight per warp
+constexpr int kDepth = 6;     // group steps in flight per warp (bitplane, NVFP4)
+constexpr int kDepthW4 = 8;   // W4: groups in flight per warp, consumed and refilled two at a time
 constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
 constexpr size_t kSmemTarget = 110 * 1024;  // two CTAs per SM
 
@@ -49,6 +51,10 @@ struct FfnArgs {
 };
 
 template <int FMT>
+__host__ __device__ constexpr int depth_of() {
+  return FMT == MOE_FMT_W4G128 ? kDepthW4 : kDepth;
+}
+template <int FMT>
 __host__ __device__ inline int slot_bytes_of() {  // one group step of one unit
   return FMT == MOE_FMT_BITPLANE8 ? 8 * kRows * 16 : (FMT == MOE_FMT_NVFP4 ? kRows * 64 + kRows * 8 : kRows * 64);
 }
@@ -66,6 +72,10 @@ MOE_DEVICE void cp_async8(void* dst, const void* src) {
 }
 MOE_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 MOE_DEVICE void cp_async_wait_depth() { asm volatile("cp.async.wait_group %0;" ::"n"(kDepth - 1) : "memory"); }
+template <int N>
+MOE_DEVICE void cp_async_wait_n() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 MOE_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- group steps
@@ -74,44 +84,47 @@ MOE_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: 
 // xv[nt][m] holds the pre-paired activations of word m of the slice for token column g
 // of tile nt; X[nt][j] the group sum of the activations of token 2c+j of tile nt.
 
-// INT4: nibbles j and j+4 of a word become one bf16x2 of (128 + u) with one shift and one
-// LOP3; the activations were paired (j, j+4) when staged.  The MMA sums (q + 136) * x onto
-// an accumulator seeded with -136 * sum(x) (the staged group sums), so after the group it
-// holds sum q * x and one FMA applies the row's scale.
+// INT4, fp16 route.  For a word w (element j of the word at nibble j)
+//   (w & 0x000F000F) | 0x64006400 = fp16 (1024 + u0, 1024 + u4)
+//   (w & 0x00F000F0) | 0x64006400 = fp16 (1024 + 16 u1, 1024 + 16 u5)
+// and the same on w >> 8 for (u2, u6) and (16 u3, 16 u7): one shift and four LOP3 per
+// eight weights.  The activations were staged as fp16 x/16 opposite the first kind and
+// x/256 opposite the second, so each product is (1032 + q) x/16 or (72 + q) x/16 (q = u - 8);
+// the accumulator starts at the staged seed -(1032 sum x/16 + 1152 sum x/256) of the
+// group and ends at sum q x/16, scaled by 16 s into the row's sum.
 template <bool TWO>
-MOE_DEVICE void w4_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa, float sb, const float (&X)[2][2],
-                         float (&acc)[2][4]) {
+MOE_DEVICE void w4h_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa16, float sb16,
+                          const float (&S)[2][2], float (&acc)[2][4]) {
   const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
   const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
-  constexpr uint32_t kMagic = 0x43004300u;  // bf16 (128, 128)
+  constexpr uint32_t kM = 0x64006400u;  // fp16 (1024, 1024)
   constexpr int NT = TWO ? 2 : 1;
   float t[2][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    t[nt][0] = t[nt][2] = -136.f * X[nt][0];
-    t[nt][1] = t[nt][3] = -136.f * X[nt][1];
+    t[nt][0] = t[nt][2] = S[nt][0];
+    t[nt][1] = t[nt][3] = S[nt][1];
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    uint32_t pa[4], pb[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      pa[j] = ((wa_[m] >> (4 * j)) & 0x000F000Fu) | kMagic;
-      pb[j] = ((wb_[m] >> (4 * j)) & 0x000F000Fu) | kMagic;
-    }
+    const uint32_t ah = wa_[m] >> 8, bh = wb_[m] >> 8;
+    const uint32_t pa0 = (wa_[m] & 0x000F000Fu) | kM, pa1 = (wa_[m] & 0x00F000F0u) | kM;
+    const uint32_t pa2 = (ah & 0x000F000Fu) | kM, pa3 = (ah & 0x00F000F0u) | kM;
+    const uint32_t pb0 = (wb_[m] & 0x000F000Fu) | kM, pb1 = (wb_[m] & 0x00F000F0u) | kM;
+    const uint32_t pb2 = (bh & 0x000F000Fu) | kM, pb3 = (bh & 0x00F000F0u) | kM;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint4 xx = xv[nt][m];
-      mma_bf16(t[nt], pa[0], pb[0], pa[1], pb[1], xx.x, xx.y);
-      mma_bf16(t[nt], pa[2], pb[2], pa[3], pb[3], xx.z, xx.w);
+      mma_f16(t[nt], pa0, pb0, pa1, pb1, xx.x, xx.y);
+      mma_f16(t[nt], pa2, pb2, pa3, pb3, xx.z, xx.w);
     }
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    acc[nt][0] = fmaf(sa, t[nt][0], acc[nt][0]);
-    acc[nt][1] = fmaf(sa, t[nt][1], acc[nt][1]);
-    acc[nt][2] = fmaf(sb, t[nt][2], acc[nt][2]);
-    acc[nt][3] = fmaf(sb, t[nt][3], acc[nt][3]);
+    acc[nt][0] = fmaf(sa16, t[nt][0], acc[nt][0]);
+    acc[nt][1] = fmaf(sa16, t[nt][1], acc[nt][1]);
+    acc[nt][2] = fmaf(sb16, t[nt][2], acc[nt][2]);
+    acc[nt][3] = fmaf(sb16, t[nt][3], acc[nt][3]);
   }
 }
 
@@ -222,7 +235,52 @@ MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const 
   }
 }
 
-// ---------------------------------------------------------------- one unit
+// ---------------------------------------------------------------- one W4 unit
+// Streams the warp's W4 unit two groups per step: waits for groups G, G+1, computes them,
+// and refills their slots with groups G + kDepthW4, G + kDepthW4 + 1 (one commit group per
+// step).  Per-lane addresses are formed once.
+template <bool TWO, class Issue>
+MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* wscale, const uint8_t* xbuf,
+                          const float* xsum, int GK, int g, int c, int nvalid, Issue&& issue, float (&acc)[2][4]) {
+  constexpr int NT = TWO ? 2 : 1;
+  constexpr int D = kDepthW4;
+  const uint8_t* xr[2] = {xbuf + size_t(g) * a.x_stride + c * 16, xbuf + size_t(8 + g) * a.x_stride + c * 16};
+  const bool live[2] = {g < nvalid, 8 + g < nvalid};
+  const float* sr[2][2] = {{xsum + (2 * c) * GK, xsum + (2 * c + 1) * GK},
+                           {xsum + (8 + 2 * c) * GK, xsum + (8 + 2 * c + 1) * GK}};
+  const uint16_t* wsa = wscale + g * GK;
+  const uint16_t* wsb = wscale + (g + 8) * GK;
+  const uint8_t* wl = wsm + g * 64 + c * 16;
+  for (int G = 0; G < GK; G += 2) {
+    cp_async_wait_n<D / 2 - 1>();
+    __syncwarp();  // every lane's copies of groups G, G+1 have landed
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int GG = G + h;
+      if (GG < GK) {
+        uint4 xv[2][4];
+        float S[2][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            xv[nt][m] = live[nt] ? *reinterpret_cast<const uint4*>(xr[nt] + GG * 256 + m * 64) : make_uint4(0, 0, 0, 0);
+          S[nt][0] = sr[nt][0][GG];
+          S[nt][1] = sr[nt][1][GG];
+        }
+        const uint8_t* wr = wl + (GG & (D - 1)) * 1024;
+        w4h_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
+                       16.f * bf16_bits_to_float(wsa[GG]), 16.f * bf16_bits_to_float(wsb[GG]), S, acc);
+      }
+    }
+    __syncwarp();  // every lane is done with these slots before they are refilled
+    if (G + D < GK) issue(G + D);
+    if (G + D + 1 < GK) issue(G + D + 1);
+    cp_async_commit();
+  }
+}
+
+// ---------------------------------------------------------------- one unit (bitplane, NVFP4)
 // Streams the warp's unit: for G = 0 .. GK-1, waits for group G's slot, computes it
 // against the staged activations of one (TWO = false) or two n8 token tiles, and refills
 // the slot with group G + kDepth.
@@ -252,11 +310,7 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t
         X[nt][1] = xsum[(nt * 8 + 2 * c + 1) * GK + G];
       }
     }
-    if (FMT == MOE_FMT_W4G128) {
-      const uint8_t* wr = sl + g * 64 + c * 16;
-      w4_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
-                    bf16_bits_to_float(wscale[g * GK + G]), bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
-    } else if (FMT == MOE_FMT_BITPLANE8) {
+    if (FMT == MOE_FMT_BITPLANE8) {
       bp_group<TWO>(sl + g * 16 + c * 4, nplanes, xv, bt, bf16_bits_to_float(wscale[g * GK + G]),
                     bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
     } else {
@@ -293,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
   float* xsum = reinterpret_cast<float*>(smem + a.off_xsum);
   int* sbits = reinterpret_cast<int*>(smem + a.off_bits);
   uint8_t* wsm = smem + size_t(warp) * a.warp_bytes;  // this warp's ring (+ scales)
-  uint16_t* wscale = reinterpret_cast<uint16_t*>(wsm + kDepth * a.slot_bytes);
+  uint16_t* wscale = reinterpret_cast<uint16_t*>(wsm + depth_of<FMT>() * a.slot_bytes);
 
   auto wrow = [&](int i) -> int {  // expert-matrix row of unit row i
     if (MODE == kGateUp) return (i < 8) ? (8 * rt + i) : (a.I + 8 * rt + i - 8);
@@ -335,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
       nplanes = min(8, nplanes);
     }
     auto issue = [&](int G) {  // copy group G of the unit into ring slot G % kDepth
-      uint8_t* dst = wsm + (G % kDepth) * a.slot_bytes;
+      uint8_t* dst = wsm + (G % depth_of<FMT>()) * a.slot_bytes;
       if (FMT == MOE_FMT_BITPLANE8) {
         const int i = lane & 15;
         for (int p = lane >> 4; p < nplanes; p += 2)
@@ -349,9 +403,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
     };
     // start this warp's weight stream before staging activations (the two overlap)
     if (has_unit) {
-      for (int G = 0; G < kDepth; ++G) {
-        if (G < GK) issue(G);
-        cp_async_commit();
+      if (FMT == MOE_FMT_W4G128) {  // two groups per commit group
+        for (int G = 0; G < kDepthW4; G += 2) {
+          if (G < GK) issue(G);
+          if (G + 1 < GK) issue(G + 1);
+          cp_async_commit();
+        }
+      } else {
+        for (int G = 0; G < kDepth; ++G) {
+          if (G < GK) issue(G);
+          cp_async_commit();
+        }
       }
       if (FMT != MOE_FMT_NVFP4) {  // the unit's 16 rows x GK scales
         const uint16_t* sb = static_cast<const uint16_t*>(a.s);
@@ -388,14 +450,26 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
         }
         uint32_t O[16];
         if (FMT == MOE_FMT_W4G128) {
+          // word m: fp16 (x0, x4)/16, (x1, x5)/256, (x2, x6)/16, (x3, x7)/256, and the seed
+          // -(1032 * sum of the /16 values + 1152 * sum of the /256 values)
+          float lo = 0.f, hi = 0.f;
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {  // word m: (x0,x4), (x1,x5), (x2,x6), (x3,x7)
+          for (int m = 0; m < 4; ++m) {
             const uint32_t r0 = R[4 * m], r1 = R[4 * m + 1], r2 = R[4 * m + 2], r3 = R[4 * m + 3];
-            O[4 * m] = __byte_perm(r0, r2, 0x5410);
-            O[4 * m + 1] = __byte_perm(r0, r2, 0x7632);
-            O[4 * m + 2] = __byte_perm(r1, r3, 0x5410);
-            O[4 * m + 3] = __byte_perm(r1, r3, 0x7632);
+            const __half2 h0 = __floats2half2_rn(bf16_lo(r0) * 0.0625f, bf16_lo(r2) * 0.0625f);
+            const __half2 h1 = __floats2half2_rn(bf16_hi(r0) * 0.00390625f, bf16_hi(r2) * 0.00390625f);
+            const __half2 h2 = __floats2half2_rn(bf16_lo(r1) * 0.0625f, bf16_lo(r3) * 0.0625f);
+            const __half2 h3 = __floats2half2_rn(bf16_hi(r1) * 0.00390625f, bf16_hi(r3) * 0.00390625f);
+            O[4 * m] = *reinterpret_cast<const uint32_t*>(&h0);
+            O[4 * m + 1] = *reinterpret_cast<const uint32_t*>(&h1);
+            O[4 * m + 2] = *reinterpret_cast<const uint32_t*>(&h2);
+            O[4 * m + 3] = *reinterpret_cast<const uint32_t*>(&h3);
+            const float2 f0 = __half22float2(h0), f1 = __half22float2(h1), f2 = __half22float2(h2),
+                         f3 = __half22float2(h3);
+            lo += (f0.x + f0.y) + (f2.x + f2.y);
+            hi += (f1.x + f1.y) + (f3.x + f3.y);
           }
+          ssum = -1032.f * lo - 1152.f * hi;
         } else if (FMT == MOE_FMT_BITPLANE8) {
 #pragma unroll
           for (int s = 0; s < 8; ++s) {  // step s: (x_2s, x_2s+16), (x_2s+1, x_2s+17)
@@ -414,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
             for (int i = 0; i < 16; ++i) O[i] = R[i];
           }
         }
-        if (FMT != MOE_FMT_NVFP4) {
+        if (FMT == MOE_FMT_BITPLANE8) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) ssum += bf16_lo(R[i]) + bf16_hi(R[i]);
         }
@@ -453,10 +527,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    if (two)
+    if (FMT == MOE_FMT_W4G128) {
+      if (two)
+        stream_w4<true>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, issue, acc);
+      else
+        stream_w4<false>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, issue, acc);
+    } else if (two) {
       stream_unit<FMT, true>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, nplanes, bt, issue, acc);
-    else
+    } else {
       stream_unit<FMT, false>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, nplanes, bt, issue, acc);
+    }
     cp_async_wait_all();
 
     // ---- epilogue: C fragment = rows g / g+8, tokens 2c, 2c+1 of each n8 tile
@@ -500,7 +580,7 @@ static bool plan(FfnArgs& a) {
   const int K = a.K, GK = K / 128;
   a.slot_bytes = slot_bytes_of<FMT>();
   const int scale_bytes = (FMT == MOE_FMT_NVFP4) ? 0 : int(align256(size_t(kRows) * GK * 2));
-  a.warp_bytes = int(align256(size_t(kDepth) * a.slot_bytes + scale_bytes));
+  a.warp_bytes = int(align256(size_t(depth_of<FMT>()) * a.slot_bytes + scale_bytes));
   a.x_stride = stride_16B(K * 2);
   const size_t fixed = size_t(kWarps) * a.warp_bytes + align256(size_t(kMaxTok) * GK * 4) + 256;
   const size_t room = fixed < kSmemTarget ? kSmemTarget - fixed : 0;
