@@ -401,8 +401,37 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
         if (FMT == MOE_FMT_NVFP4 && lane < 16) cp_async8(dst + kRows * 64 + lane * 8, sbA + G * 8);
       }
     };
-    // start this warp's weight stream before staging activations (the two overlap)
+    // start this warp's weight stream before staging activations (the two overlap); the
+    // unit's 16 rows x GK scales travel in the first commit group
     if (has_unit) {
+      if (FMT != MOE_FMT_NVFP4) {
+        const uint16_t* sb = static_cast<const uint16_t*>(a.s);
+        if ((GK & 7) == 0) {  // whole 16-byte chunks per row
+          const int cpr = GK / 8;
+          for (int idx = lane; idx < kRows * cpr; idx += 32) {
+            const int i = idx / cpr, ch = idx - i * cpr;
+            cp_async16(wscale + i * GK + ch * 8, sb + (size_t(e) * a.N + wrow(i)) * GK + ch * 8);
+          }
+        } else {  // batched loads: eight in flight per lane
+          const int n = kRows * GK;
+          for (int base = 0; base < n; base += 32 * 8) {
+            uint16_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int idx = base + u * 32 + lane;
+              if (idx < n) {
+                const int i = idx / GK, gg = idx - i * GK;
+                v[u] = sb[(size_t(e) * a.N + wrow(i)) * GK + gg];
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int idx = base + u * 32 + lane;
+              if (idx < n) wscale[idx] = v[u];
+            }
+          }
+        }
+      }
       if (FMT == MOE_FMT_W4G128) {  // two groups per commit group
         for (int G = 0; G < kDepthW4; G += 2) {
           if (G < GK) issue(G);
@@ -413,13 +442,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
         for (int G = 0; G < kDepth; ++G) {
           if (G < GK) issue(G);
           cp_async_commit();
-        }
-      }
-      if (FMT != MOE_FMT_NVFP4) {  // the unit's 16 rows x GK scales
-        const uint16_t* sb = static_cast<const uint16_t*>(a.s);
-        for (int idx = lane; idx < kRows * GK; idx += 32) {
-          const int i = idx / GK, gg = idx - i * GK;
-          wscale[idx] = sb[(size_t(e) * a.N + wrow(i)) * GK + gg];
         }
       }
     }
