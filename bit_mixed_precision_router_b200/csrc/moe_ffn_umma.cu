@@ -13,20 +13,20 @@
 // 16 gate rows and their 16 up rows: the SwiGLU product is formed in the epilogue
 // with one lane exchange.
 // Roles inside one persistent CTA (one per SM, 512 threads):
-//   warp  0     TMA producer: per 64-wide K block, the packed weight tile (4 KiB)
-//               into an 8-stage ring and the routed rows (bf16, 128-byte swizzled
-//               K-major, one 2-D box) into a 6-stage ring.  For gate/up the rows
-//               are the tokens gathered into routed order by k_gather_rows first
-//               (one bandwidth-bound pass; gathering 4 rows per TMA instruction
-//               inside the GEMM could not feed the tensor cores);
+//   warp  0     TMA producer: per 128-wide K stage (one scale group), the packed
+//               weight tile (8 KiB) into a 4-stage ring and the routed rows (bf16,
+//               128-byte swizzled K-major, two 2-D boxes of 64 K) into a 3-stage ring.
+//               For gate/up the rows are the tokens gathered into routed order by
+//               k_gather_rows first (one bandwidth-bound pass; gathering 4 rows per TMA
+//               instruction inside the GEMM could not feed the tensor cores);
 //   warp  1     allocates tensor memory; one thread issues tcgen05.mma (kind::f16,
-//               bf16 in, fp32 accumulate), A from tensor memory, B from shared
-//               memory; tcgen05.commit releases the stages;
+//               bf16 in, fp32 accumulate), eight per stage, A from tensor memory, B
+//               from shared memory; tcgen05.commit releases the stages;
 //   warps 4-11  dequantise the weights from shared memory straight into tensor
-//               memory (tcgen05.st, 4 stages of 64 K): warp 4 + 4 s + q handles
-//               rows 32 q .. 32 q + 31 of the K blocks n with n % 2 == s, so two
-//               warps per sub-partition overlap each other's waits; the bf16
-//               weight operand never exists in shared memory;
+//               memory (tcgen05.st, 2 stages of 64 columns): warp 4 + 4 s + q handles
+//               rows 32 q .. 32 q + 31 of the stages n with n % 2 == s, so two warps
+//               per sub-partition overlap each other's waits; the bf16 weight operand
+//               never exists in shared memory;
 //   warps 12-15 drain one of the two accumulators (tcgen05.ld) while the other is
 //               being accumulated, apply SwiGLU, and store bf16 rows.
 // The work list (expert, row tile, weight tile) is built by every CTA from the
@@ -50,17 +50,20 @@ namespace {
 
 constexpr int kTM = 128;        // weight rows per tile (tensor-memory lanes)
 constexpr int kTN = 192;        // routed rows per tile (MMA N at most)
-constexpr int kKB = 64;         // K elements per block: one 128-byte swizzle row of bf16
-constexpr int kBStages = 6;     // routed-row stages in shared memory
-constexpr int kWStages = 8;     // packed-weight stages in shared memory
-constexpr int kAStages = 4;     // dequantised weight stages in tensor memory
+constexpr int kKB = 128;        // K elements per stage = one scale group: two 128-byte swizzle atoms of bf16
+constexpr int kAtomK = 64;      // K elements of one 128-byte swizzle atom
+constexpr int kBStages = 3;     // routed-row stages in shared memory
+constexpr int kWStages = 4;     // packed-weight stages in shared memory
+constexpr int kAStages = 2;     // dequantised weight stages in tensor memory (64 columns each)
 constexpr int kDeqSets = 2;     // dequantising warp sets, alternating K blocks
 constexpr int kThreadsU = 32 * (4 + 4 * kDeqSets + 4);
 constexpr int kTmemCols = 512;  // accumulators at columns 0 and 192, A stages at 384 + 32 a
 constexpr int kACol0 = 2 * kTN;
-constexpr int kBStageBytes = kTN * 128;
-constexpr int kWStageBytes = kTM * 32;  // 128 rows x 64 nibbles
-constexpr int kScaleAhead = 4;          // scale groups requested ahead by the dequantisers
+constexpr int kAtomBytes = kTN * 128;   // one swizzle atom of routed rows
+constexpr int kBStageBytes = 2 * kAtomBytes;
+constexpr int kWStageBytes = kTM * 64;  // 128 rows x 128 nibbles
+constexpr int kACols = kKB / 2;         // tensor-memory columns of one A stage
+constexpr int kScaleAhead = 4;          // scale groups (stages) requested ahead by the dequantisers
 
 constexpr int kProdWarp = 0;
 constexpr int kMmaWarp = 1;
@@ -77,7 +80,7 @@ constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffTmemSlot + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // + alignment slack; > half an SM: one CTA per SM
 static_assert(kSmemBytes > 114 * 1024 && kSmemBytes <= 227 * 1024, "shared-memory plan");
-static_assert(kACol0 + kAStages * 32 <= kTmemCols, "tensor-memory plan");
+static_assert(kACol0 + kAStages * kACols <= kTmemCols, "tensor-memory plan");
 
 constexpr int kGateUp = 0, kDown = 1;
 
@@ -328,10 +331,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           mbar_arrive_expect_tx(&fullW[sw], uint32_t(kWStageBytes));
           const uint32_t wdst = sbase + kOffW + sw * kWStageBytes;
           if (MODE == kGateUp) {
-            tma_load_2d(wdst, &tm_w, kb * 32, wr0, &fullW[sw]);
-            tma_load_2d(wdst + kWStageBytes / 2, &tm_w, kb * 32, wr1, &fullW[sw]);
+            tma_load_2d(wdst, &tm_w, kb * 64, wr0, &fullW[sw]);
+            tma_load_2d(wdst + kWStageBytes / 2, &tm_w, kb * 64, wr1, &fullW[sw]);
           } else {
-            tma_load_2d(wdst, &tm_w, kb * 32, wr0, &fullW[sw]);
+            tma_load_2d(wdst, &tm_w, kb * 64, wr0, &fullW[sw]);
           }
         }
         if (!warp_wait(&emptyB[sb], ((n / kBStages) & 1) ^ 1, a.err)) {
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(&fullB[sb], uint32_t(kBStageBytes));
           tma_load_2d(bdst, &tm_b, kb * kKB, tl.r0, &fullB[sb]);
+          tma_load_2d(bdst + kAtomBytes, &tm_b, kb * kKB + kAtomK, tl.r0, &fullB[sb]);
         }
       }
     }
@@ -366,10 +370,11 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           }
           tc_fence_after();
           const uint64_t bdesc = bdesc0 + uint64_t((sb * kBStageBytes) >> 4);
-          const uint32_t a_tmem = tmem + uint32_t(kACol0 + sa * 32);
+          const uint32_t a_tmem = tmem + uint32_t(kACol0 + sa * kACols);
 #pragma unroll
-          for (int kk = 0; kk < kKB / 16; ++kk)
-            tc_mma_ts(d_tmem, a_tmem + kk * 8, bdesc + uint64_t(2 * kk), idesc, (kb | kk) != 0);
+          for (int kk = 0; kk < kKB / 16; ++kk)  // atom kk / 4, 32 bytes per K=16 step inside it
+            tc_mma_ts(d_tmem, a_tmem + kk * 8, bdesc + uint64_t((kk >> 2) * (kAtomBytes >> 4) + 2 * (kk & 3)),
+                      idesc, (kb | kk) != 0);
           tc_commit(&emptyB[sb]);
           tc_commit(&emptyA[sa]);
         }
@@ -390,65 +395,72 @@ __global__ void __launch_bounds__(kThreadsU, 1)
                                        : quarter * 32 + lane;
     const int my_items = blockIdx.x < n_items ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
     const int total = my_items * KB;
-    // scales: one bf16 per 128 K (every other block), requested kScaleAhead groups ahead
+    // scales: one bf16 per stage (128 K), requested kScaleAhead of this set's stages ahead;
+    // set s converts stages n = 2 m + s (m = 0, 1, ...)
+    const int my_stages = (total - set + 1) / 2;
     int s_li = -1;
     const uint16_t* s_row = nullptr;
-    auto scale_at = [&](int g2) -> uint32_t {  // g2 = flat index of a 128-wide group
-      const int li = (2 * g2) / KB, grp = g2 - li * (KB / 2);
+    auto scale_at = [&](int m) -> uint32_t {
+      const int n = 2 * m + set;
+      const int li = n / KB, grp = n - li * KB;
       if (li != s_li) {
         s_li = li;
         const Tile tl = tile_of(int(blockIdx.x) + li * int(gridDim.x), pre, E, a.wtiles, a.offsets);
-        int n;
-        if (MODE == kGateUp) n = (srow < 64) ? tl.wt * 64 + srow : a.I + tl.wt * 64 + (srow - 64);
-        else n = tl.wt * kTM + srow;
-        s_row = a.s + (size_t(tl.e) * a.n_rows + n) * KG;
+        int r;
+        if (MODE == kGateUp) r = (srow < 64) ? tl.wt * 64 + srow : a.I + tl.wt * 64 + (srow - 64);
+        else r = tl.wt * kTM + srow;
+        s_row = a.s + (size_t(tl.e) * a.n_rows + r) * KG;
       }
       return s_row[grp];
     };
     uint32_t sring[kScaleAhead];
-    const int total_g = total / 2;
 #pragma unroll
-    for (int q = 0; q < kScaleAhead; ++q) sring[q] = (q < total_g) ? scale_at(q) : 0u;
+    for (int q = 0; q < kScaleAhead; ++q) sring[q] = (q < my_stages) ? scale_at(q) : 0u;
     bool ok = true;
-    for (int g0 = 0; g0 < total_g && ok; g0 += kScaleAhead) {
+    for (int m0 = 0; m0 < my_stages && ok; m0 += kScaleAhead) {
 #pragma unroll
       for (int q = 0; q < kScaleAhead; ++q) {
-        const int g2 = g0 + q;
-        if (g2 >= total_g) break;
+        const int m = m0 + q;
+        if (m >= my_stages) break;
         const uint32_t sv = sring[q];
-        if (g2 + kScaleAhead < total_g) sring[q] = scale_at(g2 + kScaleAhead);
+        if (m + kScaleAhead < my_stages) sring[q] = scale_at(m + kScaleAhead);
         const uint32_t s2 = sv | (sv << 16);
-        {
-          const int n = 2 * g2 + set;
-          const int sw = n % kWStages, sa = n % kAStages;
-          if (!warp_wait(&fullW[sw], (n / kWStages) & 1, a.err)) {
-            ok = false;
-            break;
-          }
-          const uint32_t wrow = sbase + kOffW + sw * kWStageBytes + srow * 32;
-          const uint4 w0 = lds128(wrow), w1 = lds128(wrow + 16);
-          const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          uint32_t v[32];
+        const int n = 2 * m + set;
+        const int sw = n % kWStages, sa = n % kAStages;
+        if (!warp_wait(&fullW[sw], (n / kWStages) & 1, a.err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t wrow = sbase + kOffW + sw * kWStageBytes + srow * 64;
+        uint4 wq[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) wq[h] = lds128(wrow + 16 * h);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&emptyW[sw]);
+        uint32_t v[2][32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t words[8] = {wq[2 * h].x,     wq[2 * h].y,     wq[2 * h].z,     wq[2 * h].w,
+                                     wq[2 * h + 1].x, wq[2 * h + 1].y, wq[2 * h + 1].z, wq[2 * h + 1].w};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             uint32_t p[4];
             w4_word_pairs(words[i], p);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
+            for (int j = 0; j < 4; ++j) v[h][4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&emptyW[sw]);
-          if (!warp_wait(&emptyA[sa], ((n / kAStages) & 1) ^ 1, a.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          tmem_st32(tmem + lane_base + uint32_t(kACol0 + sa * 32), v);
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&fullA[sa]);
         }
+        if (!warp_wait(&emptyA[sa], ((n / kAStages) & 1) ^ 1, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem + lane_base + uint32_t(kACol0 + sa * kACols), v[0]);
+        tmem_st32(tmem + lane_base + uint32_t(kACol0 + sa * kACols + 32), v[1]);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&fullA[sa]);
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -618,10 +630,10 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
   if (err != cudaSuccess) return err;
   CUtensorMap tb, tw;
   // gate/up: routed token rows in one box per stage; weight boxes of 64 gate and 64 up rows
-  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs, uint64_t(H), uint64_t(P), uint64_t(H) * 2, kKB, kTN,
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs, uint64_t(H), uint64_t(P), uint64_t(H) * 2, kAtomK, kTN,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w13, uint64_t(H) / 2, uint64_t(E) * 2 * I,
-                   uint64_t(H) / 2, 32, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+                   uint64_t(H) / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   a.K = H;
   a.n_rows = 2 * I;
@@ -632,9 +644,9 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
   err = launch_umma_one<kGateUp>(tb, tw, a, st);
   if (err != cudaSuccess) return err;
   // down: h rows in one box per stage; weight boxes of 128 rows
-  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hbuf, uint64_t(I), uint64_t(P), uint64_t(I) * 2, kKB,
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hbuf, uint64_t(I), uint64_t(P), uint64_t(I) * 2, kAtomK,
                    kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 32,
+      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 64,
                    kTM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   a.K = I;
