@@ -5,6 +5,8 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -117,6 +119,23 @@ MOE_DEVICE uint4 ldg_nc_v4(const void* p) {
 }
 
 MOE_DEVICE float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// ---------------------------------------------------------------- NVFP4 element conversions
+// byte = two E2M1 codes (element 2i in the low nibble) -> fp16x2 (low half = element 2i)
+MOE_DEVICE uint32_t e2m1x2_to_h2(uint32_t byte) {
+  const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
+  return uint32_t(r.x) | (uint32_t(r.y) << 16);
+}
+// E4M3 code -> fp16x2 (the value in both halves)
+MOE_DEVICE uint32_t e4m3_to_h2(uint32_t byte) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(byte), __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.x) << 16);
+}
+MOE_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 
 }  // namespace moe
 

@@ -14,9 +14,6 @@
 // nibble / bit / FP4 -> fp16 or bf16 in registers, mma.sync m16n8k16 with the tokens on N.
 // W4 takes two groups per wait and converts nibbles to fp16 against activations staged
 // in fp16 (see w4h_group).  Expert weights are read from HBM once per token chunk.
-#include <cuda_fp4.h>
-#include <cuda_fp8.h>
-
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -194,20 +191,6 @@ MOE_DEVICE void bp_group(const uint8_t* pl, int nplanes, const uint4 (&xv)[2][4]
 // NVFP4: byte i of a word holds elements 2i (low nibble) and 2i+1; the hardware converts
 // the pair to fp16 and the E4M3 block scale multiplies it in fp16 (exact); activations
 // are fp16 * 2^-8 in natural pairs.
-MOE_DEVICE uint32_t e2m1x2_to_h2(uint32_t byte) {
-  const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
-  return uint32_t(r.x) | (uint32_t(r.y) << 16);
-}
-MOE_DEVICE uint32_t e4m3_to_h2(uint32_t byte) {
-  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(byte), __NV_E4M3);
-  return uint32_t(h.x) | (uint32_t(h.x) << 16);
-}
-MOE_DEVICE uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
 template <bool TWO>
 MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const uint4 (&xv)[2][4],
                           float (&acc)[2][4]) {

@@ -90,8 +90,10 @@ struct UmmaArgs {
   int n_rows;                // rows of one expert's weight matrix (2I or H)
   const int32_t* offsets;    // [E+1]
   const int32_t* sorted_pair;
-  const uint16_t* s;         // bf16 scales [E][n_rows][K/128]
-  uint16_t* out;             // gate/up: h [P][I]; down: y [P][H]
+  const uint16_t* s;         // W4: bf16 scales [E][n_rows][K/128]
+  const uint8_t* bs;         // NVFP4: E4M3 block scales [E][n_rows][K/16]
+  const float* gs;           // NVFP4: per-expert fp32 scale of this matrix [E]
+  uint16_t* out;             // gate/up: h [P][I] (bf16; NVFP4: fp16 h/256); down: y [P][H] bf16
   int out_ld;
   unsigned* err;
 };
@@ -188,9 +190,12 @@ MOE_DEVICE uint64_t sw128_desc(uint32_t saddr) {
   d |= uint64_t(2) << 61;             // 128-byte swizzle
   return d;
 }
-// Instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M = 128.
-MOE_DEVICE uint32_t idesc_bf16(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTM >> 4) << 24);
+// Instruction descriptor: fp32 accumulate, A and B both bf16 (W4) or both fp16 (NVFP4),
+// both K-major, M = 128.
+template <int FMT>
+MOE_DEVICE uint32_t idesc_mma(int n) {
+  const uint32_t ab = (FMT == MOE_FMT_NVFP4) ? 0u : 1u;  // 0 = f16, 1 = bf16
+  return (1u << 4) | (ab << 7) | (ab << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTM >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- W4 dequant
@@ -238,7 +243,7 @@ MOE_DEVICE Tile tile_of(int item, const int* pre, int E, int wtiles, const int32
   return tl;
 }
 
-template <int MODE>
+template <int FMT, int MODE>
 __global__ void __launch_bounds__(kThreadsU, 1)
     k_ffn_umma(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w, UmmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         const int ab = it & 1;
         if (!mbar_wait(&accEmpty[ab], ((it >> 1) & 1) ^ 1, a.err)) break;
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16((tl.nrows + 15) & ~15);
+        const uint32_t idesc = idesc_mma<FMT>((tl.nrows + 15) & ~15);
         const uint32_t d_tmem = tmem + uint32_t(ab * kTN);
         for (int kb = 0; kb < KB; ++kb, ++n) {
           const int sb = n % kBStages, sa = n % kAStages;
@@ -398,9 +403,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     // scales: one bf16 per stage (128 K), requested kScaleAhead of this set's stages ahead;
     // set s converts stages n = 2 m + s (m = 0, 1, ...)
     const int my_stages = (total - set + 1) / 2;
+    // W4: the stage's bf16 group scale; NVFP4: the stage's eight E4M3 block scales
     int s_li = -1;
-    const uint16_t* s_row = nullptr;
-    auto scale_at = [&](int m) -> uint32_t {
+    size_t s_row = 0;  // index of this lane's weight row in [E * n_rows]
+    auto scale_at = [&](int m) -> uint2 {
       const int n = 2 * m + set;
       const int li = n / KB, grp = n - li * KB;
       if (li != s_li) {
@@ -409,22 +415,22 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         int r;
         if (MODE == kGateUp) r = (srow < 64) ? tl.wt * 64 + srow : a.I + tl.wt * 64 + (srow - 64);
         else r = tl.wt * kTM + srow;
-        s_row = a.s + (size_t(tl.e) * a.n_rows + r) * KG;
+        s_row = size_t(tl.e) * a.n_rows + r;
       }
-      return s_row[grp];
+      if (FMT == MOE_FMT_NVFP4) return *reinterpret_cast<const uint2*>(a.bs + s_row * size_t(KG * 8) + grp * 8);
+      return make_uint2(a.s[s_row * KG + grp], 0u);
     };
-    uint32_t sring[kScaleAhead];
+    uint2 sring[kScaleAhead];
 #pragma unroll
-    for (int q = 0; q < kScaleAhead; ++q) sring[q] = (q < my_stages) ? scale_at(q) : 0u;
+    for (int q = 0; q < kScaleAhead; ++q) sring[q] = (q < my_stages) ? scale_at(q) : make_uint2(0u, 0u);
     bool ok = true;
     for (int m0 = 0; m0 < my_stages && ok; m0 += kScaleAhead) {
 #pragma unroll
       for (int q = 0; q < kScaleAhead; ++q) {
         const int m = m0 + q;
         if (m >= my_stages) break;
-        const uint32_t sv = sring[q];
+        const uint2 sv = sring[q];
         if (m + kScaleAhead < my_stages) sring[q] = scale_at(m + kScaleAhead);
-        const uint32_t s2 = sv | (sv << 16);
         const int n = 2 * m + set;
         const int sw = n % kWStages, sa = n % kAStages;
         if (!warp_wait(&fullW[sw], (n / kWStages) & 1, a.err)) {
@@ -438,16 +444,35 @@ __global__ void __launch_bounds__(kThreadsU, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&emptyW[sw]);
         uint32_t v[2][32];
+        if (FMT == MOE_FMT_NVFP4) {
+          // byte c of the row's 64 = elements 2c, 2c+1 (column c); 16 elements per block scale,
+          // e2m1 * e4m3 is exact in fp16
+          uint32_t sb2[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t words[8] = {wq[2 * h].x,     wq[2 * h].y,     wq[2 * h].z,     wq[2 * h].w,
-                                     wq[2 * h + 1].x, wq[2 * h + 1].y, wq[2 * h + 1].z, wq[2 * h + 1].w};
+          for (int b = 0; b < 8; ++b) sb2[b] = e4m3_to_h2(((b < 4 ? sv.x : sv.y) >> (8 * (b & 3))) & 0xFFu);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint32_t p[4];
-            w4_word_pairs(words[i], p);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t words[8] = {wq[2 * h].x,     wq[2 * h].y,     wq[2 * h].z,     wq[2 * h].w,
+                                       wq[2 * h + 1].x, wq[2 * h + 1].y, wq[2 * h + 1].z, wq[2 * h + 1].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[h][4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                v[h][4 * i + j] = hmul2(e2m1x2_to_h2((words[i] >> (8 * j)) & 0xFFu), sb2[4 * h + (i >> 1)]);
+          }
+        } else {
+          const uint32_t s2 = sv.x | (sv.x << 16);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t words[8] = {wq[2 * h].x,     wq[2 * h].y,     wq[2 * h].z,     wq[2 * h].w,
+                                       wq[2 * h + 1].x, wq[2 * h + 1].y, wq[2 * h + 1].z, wq[2 * h + 1].w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              uint32_t p[4];
+              w4_word_pairs(words[i], p);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) v[h][4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
+            }
           }
         }
         if (!warp_wait(&emptyA[sa], ((n / kAStages) & 1) ^ 1, a.err)) {
@@ -473,6 +498,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int ab = it & 1;
       if (!warp_wait(&accFull[ab], (it >> 1) & 1, a.err)) break;
       tc_fence_after();
+      // NVFP4: the accumulator holds sum (e2m1 * e4m3) * x / 256
+      const float post = (FMT == MOE_FMT_NVFP4) ? 256.f * a.gs[tl.e] : 1.f;
       for (int c0 = 0; c0 < tl.nrows; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + uint32_t(ab * kTN + c0), v);
@@ -482,15 +509,19 @@ __global__ void __launch_bounds__(kThreadsU, 1)
           uint16_t* o = a.out + size_t(tl.r0 + c0) * a.out_ld + tl.wt * kTM + quarter * 32 + lane;
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (c < nc) o[size_t(c) * a.out_ld] = float_to_bf16_bits(__uint_as_float(v[c]));
+            if (c < nc) o[size_t(c) * a.out_ld] = float_to_bf16_bits(__uint_as_float(v[c]) * post);
         } else {
           // lane l < 16 holds gate column i, lane l + 16 the up value of the same i
           uint16_t* o = a.out + size_t(tl.r0 + c0) * a.out_ld + tl.wt * 64 + quarter * 16 + (lane & 15);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float mine = __uint_as_float(v[c]);
+            const float mine = __uint_as_float(v[c]) * post;
             const float up = __shfl_xor_sync(0xffffffffu, mine, 16);
-            if (lane < 16 && c < nc) o[size_t(c) * a.out_ld] = float_to_bf16_bits(silu(mine) * up);
+            if (lane < 16 && c < nc) {
+              const float hv = silu(mine) * up;
+              o[size_t(c) * a.out_ld] = (FMT == MOE_FMT_NVFP4) ? __half_as_ushort(__float2half_rn(hv * (1.f / 256.f)))
+                                                                : float_to_bf16_bits(hv);
+            }
           }
         }
       }
@@ -510,6 +541,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
 
 // xs[r] = x[sorted_pair[r] / k]: the token rows in routed order; one warp per row,
 // 16 bytes per lane per step, four steps in flight.
+// NVFP4: the rows are written as fp16 x/256 (the GEMM's B operand type).
+template <int FMT>
 __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_pair,
                                                      int P, int k, int row16, uint4* __restrict__ xs) {
   const int lane = threadIdx.x & 31;
@@ -527,7 +560,20 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = c0 + 32 * u + lane;
-        if (c < row16) dst[c] = v[u];
+        if (c < row16) {
+          if (FMT == MOE_FMT_NVFP4) {
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const __half2 hh = __floats2half2_rn(bf16_lo(w[i]) * (1.f / 256.f), bf16_hi(w[i]) * (1.f / 256.f));
+              o[i] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+            dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+          } else {
+            dst[c] = v[u];
+          }
+        }
       }
     }
   }
@@ -575,7 +621,7 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int MODE>
+template <int FMT, int MODE>
 cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const UmmaArgs& a, cudaStream_t st) {
   static bool raised[128] = {};
   int dev = 0;
@@ -583,13 +629,13 @@ cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const 
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!raised[dev]) {
     const cudaError_t err =
-        cudaFuncSetAttribute(k_ffn_umma<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(k_ffn_umma<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
     raised[dev] = true;
   }
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  k_ffn_umma<MODE><<<nsm, kThreadsU, kSmemBytes, st>>>(tb, tw, a);
+  k_ffn_umma<FMT, MODE><<<nsm, kThreadsU, kSmemBytes, st>>>(tb, tw, a);
   return cudaGetLastError();
 }
 
@@ -598,19 +644,19 @@ cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const 
 // At 32 or more rows per expert on average, the tensor-core GEMM (weights
 // dequantised once per 192 rows) beats streaming the weights once per 16 rows.
 bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt) {
-  return fmt == MOE_FMT_W4G128 && T * k >= 32 * E;
+  return (fmt == MOE_FMT_W4G128 || fmt == MOE_FMT_NVFP4) && T * k >= 32 * E;
 }
 
 static size_t align256u(size_t b) { return (b + 255) / 256 * 256; }
 size_t umma_h_bytes(int64_t T, int64_t I, int64_t k) { return align256u(size_t(T * k * I * 2)); }
-// h [P][I] bf16, then the routed token rows [P][H] bf16
+// h [P][I], then the routed token rows [P][H] (2-byte elements: bf16 for W4, fp16/256 for NVFP4)
 size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k) {
   return umma_h_bytes(T, I, k) + align256u(size_t(T * k * H * 2));
 }
 
-cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
-                                    int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st) {
-  if (ex.fmt != MOE_FMT_W4G128) return cudaErrorInvalidValue;
+template <int FMT>
+static cudaError_t launch_umma_fmt(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H,
+                                   int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st) {
   const int P = T * k;
   UmmaArgs a{};
   a.E = E;
@@ -622,15 +668,18 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
   if (!a.err) return cudaErrorInvalidDevice;
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
+  const CUtensorMapDataType act_type =
+      (FMT == MOE_FMT_NVFP4) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   // the token rows in routed order, after h in the workspace
   uint16_t* xs = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(hbuf) + umma_h_bytes(T, I, k));
-  k_gather_rows<<<4 * nsm, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), r.sorted_pair, P, k, H / 8,
-                                         reinterpret_cast<uint4*>(xs));
+  k_gather_rows<FMT><<<4 * nsm, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), r.sorted_pair, P, k, H / 8,
+                                              reinterpret_cast<uint4*>(xs));
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   CUtensorMap tb, tw;
-  // gate/up: routed token rows in one box per stage; weight boxes of 64 gate and 64 up rows
-  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs, uint64_t(H), uint64_t(P), uint64_t(H) * 2, kAtomK, kTN,
+  // gate/up: routed token rows, two 64-K boxes per stage; weight boxes of 64 gate and 64 up
+  // rows (packed W4 words and E2M1 codes both take K/2 bytes per row)
+  if (!make_map_2d(&tb, act_type, xs, uint64_t(H), uint64_t(P), uint64_t(H) * 2, kAtomK, kTN,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w13, uint64_t(H) / 2, uint64_t(E) * 2 * I,
                    uint64_t(H) / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -639,13 +688,15 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
   a.n_rows = 2 * I;
   a.wtiles = I / 64;
   a.s = static_cast<const uint16_t*>(ex.w13_scale);
+  a.bs = static_cast<const uint8_t*>(ex.w13_scale);
+  a.gs = ex.w13_gscale;
   a.out = static_cast<uint16_t*>(hbuf);
   a.out_ld = I;
-  err = launch_umma_one<kGateUp>(tb, tw, a, st);
+  err = launch_umma_one<FMT, kGateUp>(tb, tw, a, st);
   if (err != cudaSuccess) return err;
-  // down: h rows in one box per stage; weight boxes of 128 rows
-  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hbuf, uint64_t(I), uint64_t(P), uint64_t(I) * 2, kAtomK,
-                   kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // down: h rows, two 64-K boxes per stage; weight boxes of 128 rows
+  if (!make_map_2d(&tb, act_type, hbuf, uint64_t(I), uint64_t(P), uint64_t(I) * 2, kAtomK, kTN,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 64,
                    kTM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
@@ -653,9 +704,19 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
   a.n_rows = H;
   a.wtiles = H / kTM;
   a.s = static_cast<const uint16_t*>(ex.w2_scale);
+  a.bs = static_cast<const uint8_t*>(ex.w2_scale);
+  a.gs = ex.w2_gscale;
   a.out = y_rows;
   a.out_ld = H;
-  return launch_umma_one<kDown>(tb, tw, a, st);
+  return launch_umma_one<FMT, kDown>(tb, tw, a, st);
+}
+
+cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
+                                    int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st) {
+  if (ex.fmt == MOE_FMT_W4G128)
+    return launch_umma_fmt<MOE_FMT_W4G128>(x, r, ex, T, H, I, E, k, y_rows, hbuf, st);
+  if (ex.fmt == MOE_FMT_NVFP4) return launch_umma_fmt<MOE_FMT_NVFP4>(x, r, ex, T, H, I, E, k, y_rows, hbuf, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

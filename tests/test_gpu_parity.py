@@ -185,7 +185,8 @@ def bf16_f64(b):
 
 
 # Batches with 32 or more rows per expert on average take the tensor-core GEMM
-# path (tcgen05, W4 group-128): 128-row tiles of weights and of routed rows.
+# path (tcgen05; W4 group-128 in bf16, NVFP4 in fp16): 128-row weight tiles, up to
+# 192 routed rows per tile.
 GEMM_CASES = [
     # T, H, I, E, k, zipf
     (512, 256, 128, 8, 2, False),     # ~128 rows per expert: one or two row tiles
@@ -196,17 +197,18 @@ GEMM_CASES = [
 ]
 
 
+@pytest.mark.parametrize("fmt", [FMT_W4G128, FMT_NVFP4])
 @pytest.mark.parametrize("T,H,I,E,k,zipf", GEMM_CASES)
-def test_grouped_gemm_path(moe, cuda_device, T, H, I, E, k, zipf):
+def test_grouped_gemm_path(moe, cuda_device, fmt, T, H, I, E, k, zipf):
     assert T * k >= 32 * E
     L = make_layer(3000 + T + E, T, H, I, E, k, zipf=zipf)
-    ex_o = oracle_experts(FMT_W4G128, L.w13, L.w2)
-    ex_g = moe.quantize_experts(FMT_W4G128, dev_bf16(L.w13), dev_bf16(L.w2))
+    ex_o = oracle_experts(fmt, L.w13, L.w2)
+    ex_g = moe.quantize_experts(fmt, dev_bf16(L.w13), dev_bf16(L.w2))
     out, (logits, ids, w, offsets, sp, p2r) = _route_both(moe, L, k)
     assert np.array_equal(out.sorted_pair.cpu().numpy(), sp)
     y = moe.moe_grouped_ffn(dev_bf16(L.x), out, ex_g, I, E, k)
     o = moe.moe_combine(y, out, T, k)
     moe.moe_check_device_errors()
     y_ref = grouped_ffn(L.x, offsets, sp, k, ex_o, None)
-    check_close(bf16_f64(host_bits(y)), y_ref, "y_rows (GEMM path)")
-    check_close(bf16_f64(host_bits(o)), combine(y_ref, w, p2r, None), "out (GEMM path)")
+    check_close(bf16_f64(host_bits(y)), y_ref, f"y_rows (GEMM path, fmt={fmt})")
+    check_close(bf16_f64(host_bits(o)), combine(y_ref, w, p2r, None), f"out (GEMM path, fmt={fmt})")
