@@ -51,6 +51,11 @@ PREFILL = {
     "prefill-h7168-e256": dict(T=4096, H=7168, I=2048, E=256, k=8, router="uniform", zipf=False, seed=0x5EED0005,
                                desc="one MoE FFN layer, H7168 I2048 E256 top-8, W4A16 g128 experts, "
                                     "U(-0.02, 0.02) bf16 router, 4096 fresh tokens per step"),
+    "prefill-h7168-e256-nvfp4": dict(T=4096, H=7168, I=2048, E=256, k=8, router="uniform", zipf=False,
+                                     seed=0x5EED0005, fmt="nvfp4",
+                                     desc="one MoE FFN layer, H7168 I2048 E256 top-8, NVFP4 experts (E2M1, E4M3 "
+                                          "per 16, fp32 per tensor), U(-0.02, 0.02) bf16 router, 4096 fresh "
+                                          "tokens per step"),
 }
 
 
@@ -391,17 +396,26 @@ class PrefillLayer:
         T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
         seed = cfg["seed"]
         i32, bf = dict(dtype=torch.int32, device=device), dict(dtype=torch.bfloat16, device=device)
-        w13q, w13s = torch.empty((Ee, 2 * Ii, Hh // 8), **i32), torch.empty((Ee, 2 * Ii, Hh // 128), **bf)
-        w2q, w2s = torch.empty((Ee, Hh, Ii // 8), **i32), torch.empty((Ee, Hh, Ii // 128), **bf)
+        u8, f32 = dict(dtype=torch.uint8, device=device), dict(dtype=torch.float32, device=device)
+        self.fmt = moe.FMT_NVFP4 if cfg.get("fmt") == "nvfp4" else moe.FMT_W4G128
+        if self.fmt == moe.FMT_NVFP4:
+            mk = lambda n, kk: (torch.empty((Ee, n, kk // 2), **u8), torch.empty((Ee, n, kk // 16), **u8),
+                                torch.empty((Ee,), **f32))
+        else:
+            mk = lambda n, kk: (torch.empty((Ee, n, kk // 8), **i32), torch.empty((Ee, n, kk // 128), **bf), None)
+        w13, w2 = mk(2 * Ii, Hh), mk(Hh, Ii)
         tmp = torch.empty((chunk * 2 * Ii * Hh,), **bf)
-        for (n, kk, tag, q, sc) in ((2 * Ii, Hh, synth.SEED_W13, w13q, w13s), (Hh, Ii, synth.SEED_W2, w2q, w2s)):
+        for (n, kk, tag, st) in ((2 * Ii, Hh, synth.SEED_W13, w13), (Hh, Ii, synth.SEED_W2, w2)):
             for e0 in range(0, Ee, chunk):
                 ne = min(chunk, Ee - e0)
                 t = tmp[:ne * n * kk].view(ne, n, kk)
                 moe.moe_synth_normal_bf16(t, seed + tag, 0.02, start=e0 * n * kk)
-                moe.moe_quantize_w4g128(t, q[e0:e0 + ne], sc[e0:e0 + ne])
+                if self.fmt == moe.FMT_NVFP4:
+                    moe.moe_quantize_nvfp4(t, st[0][e0:e0 + ne], st[1][e0:e0 + ne], st[2][e0:e0 + ne])
+                else:
+                    moe.moe_quantize_w4g128(t, st[0][e0:e0 + ne], st[1][e0:e0 + ne])
         del tmp
-        self.experts = moe.Experts(moe.FMT_W4G128, w13q, w13s, w2q, w2s)
+        self.experts = moe.Experts(self.fmt, w13[0], w13[1], w2[0], w2[1], w13[2], w2[2])
         self.wr = torch.empty((Ee, Hh), **bf)
         if cfg["router"] == "uniform":
             moe.moe_synth_uniform_bf16(self.wr, seed + synth.SEED_WR, -0.02, 0.02)
@@ -411,7 +425,7 @@ class PrefillLayer:
             if cfg["zipf"] else None
         self.routing = moe.Routing.empty(T, Ee, k, device)
         self.route_ws = moe.moe_route_workspace(T, Ee, k, device)
-        self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(T, Hh, Ii, Ee, k, moe.FMT_W4G128), 16),
+        self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(T, Hh, Ii, Ee, k, self.fmt), 16),
                                   dtype=torch.uint8, device=device)
         self.y_rows = torch.empty((T * k, Hh), **bf)
         self.x = torch.empty((T, Hh), **bf)
@@ -528,12 +542,13 @@ def run_prefill(args, rank, world, local):
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, "
-                                                          "N(0,0.02) bf16 weights quantised to W4A16 g128)",
+            "vs_baseline": None, "dtype": "fp16" if cfg.get("fmt") == "nvfp4" else "bf16",
+            "data": "synthetic (seeded Irwin-Hall N(0,1) activations, N(0,0.02) bf16 weights quantised to "
+                    + ("NVFP4" if cfg.get("fmt") == "nvfp4" else "W4A16 g128") + ")",
             "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,
                        "top_k": k, "parallelism": f"dp{world} (independent replicas)",
-                       "l2": "no flush: each step reads %.2f GB of expert weights, > 126 MB L2"
-                             % (Ee * (3 * Hh * Ii // 2 + 3 * Hh * Ii // 64) / 1e9)},
+                       "l2": "no flush: each step reads more than %.1f GB of expert weights, > 126 MB L2"
+                             % (Ee * 3 * Hh * Ii / 2 / 1e9)},
             "gpu_launches": PrefillLayer.kernels_per_step * K,
             "clocks": clk, "roofline": roofline, "e2e": e2e,
         }
@@ -551,10 +566,11 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
     import numpy as np
 
     import synth
-    from oracle.ffn import FMT_W4G128, Experts, moe_layer
-    from oracle.quant import quantize_w4g128
+    from oracle.ffn import FMT_NVFP4, FMT_W4G128, Experts, moe_layer
+    from oracle.quant import quantize_nvfp4, quantize_w4g128
     from oracle.routing import router_logits, topk_softmax
     T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
+    nvfp4 = cfg.get("fmt") == "nvfp4"
     x = synth.normal_bf16(seed + synth.SEED_X, tokens * Hh, 1.0).reshape(tokens, Hh)
     if cfg["router"] == "uniform":
         wr = synth.uniform_bf16(cfg["seed"] + synth.SEED_WR, Ee * Hh, -0.02, 0.02).reshape(Ee, Hh)
@@ -562,15 +578,23 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
         wr = synth.normal_bf16(cfg["seed"] + synth.SEED_WR, Ee * Hh, 0.02).reshape(Ee, Hh)
     bias = synth.zipf_rank_bias(cfg["seed"] + synth.SEED_BIAS, Ee) if cfg["zipf"] else None
     ids, _ = topk_softmax(router_logits(x, wr, bias), k)
-    w13q = np.zeros((Ee, 2 * Ii, Hh // 8), np.uint32)
-    w13s = np.zeros((Ee, 2 * Ii, Hh // 128), np.uint16)
-    w2q = np.zeros((Ee, Hh, Ii // 8), np.uint32)
-    w2s = np.zeros((Ee, Hh, Ii // 128), np.uint16)
+    if nvfp4:
+        w13q, w13s = np.zeros((Ee, 2 * Ii, Hh // 2), np.uint8), np.zeros((Ee, 2 * Ii, Hh // 16), np.uint8)
+        w2q, w2s = np.zeros((Ee, Hh, Ii // 2), np.uint8), np.zeros((Ee, Hh, Ii // 16), np.uint8)
+        w13g, w2g = np.zeros(Ee, np.float32), np.zeros(Ee, np.float32)
+    else:
+        w13q, w13s = np.zeros((Ee, 2 * Ii, Hh // 8), np.uint32), np.zeros((Ee, 2 * Ii, Hh // 128), np.uint16)
+        w2q, w2s = np.zeros((Ee, Hh, Ii // 8), np.uint32), np.zeros((Ee, Hh, Ii // 128), np.uint16)
     for e in sorted(set(ids.reshape(-1).tolist())):
-        a = quantize_w4g128(synth.normal_rows_bf16(cfg["seed"] + synth.SEED_W13, (2 * Ii, Hh), 0.02, e, 1))
-        b = quantize_w4g128(synth.normal_rows_bf16(cfg["seed"] + synth.SEED_W2, (Hh, Ii), 0.02, e, 1))
-        w13q[e], w13s[e], w2q[e], w2s[e] = a[0][0], a[1][0], b[0][0], b[1][0]
-    ex = Experts(FMT_W4G128, w13q, w13s, w2q, w2s)
+        r13 = synth.normal_rows_bf16(cfg["seed"] + synth.SEED_W13, (2 * Ii, Hh), 0.02, e, 1)
+        r2 = synth.normal_rows_bf16(cfg["seed"] + synth.SEED_W2, (Hh, Ii), 0.02, e, 1)
+        if nvfp4:
+            a, b = quantize_nvfp4(r13), quantize_nvfp4(r2)
+            w13q[e], w13s[e], w13g[e], w2q[e], w2s[e], w2g[e] = a[0][0], a[1][0], a[2][0], b[0][0], b[1][0], b[2][0]
+        else:
+            a, b = quantize_w4g128(r13), quantize_w4g128(r2)
+            w13q[e], w13s[e], w2q[e], w2s[e] = a[0][0], a[1][0], b[0][0], b[1][0]
+    ex = Experts(FMT_NVFP4, w13q, w13s, w2q, w2s, w13g, w2g) if nvfp4 else Experts(FMT_W4G128, w13q, w13s, w2q, w2s)
     t0 = time.perf_counter()
     moe_layer(x, wr, bias, ex, k, residual_bits=x)
     secs = time.perf_counter() - t0
@@ -622,7 +646,10 @@ def oracle_sample(batch: int, layers_timed: int, seed: int):
 
 
 def prefill_sample_tokens(cfg) -> int:
-    return 2 if cfg["H"] > 4096 else 32  # bounded: a few to about 30 s of oracle work
+    # bounded: a few to about 30 s of oracle work (the NVFP4 oracle decodes element by element)
+    if cfg.get("fmt") == "nvfp4":
+        return 1
+    return 2 if cfg["H"] > 4096 else 32
 
 
 def cpu_baseline_prefill(cfg, seed: int):
