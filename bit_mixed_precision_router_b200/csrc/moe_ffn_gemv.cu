@@ -5,7 +5,9 @@
 //            MMA fragment gives gate and up of 8 intermediate rows, so SwiGLU runs in
 //            the epilogue);
 //   down:    rows 0..15 = down rows 16t..16t+15.
-// One CTA = one routed expert x 8 warps, each warp owning whole units.  The expert's
+// One CTA = one routed expert x 4 warps, each warp owning one 16-row unit; four CTAs per
+// SM (small CTAs start at different times, so one CTA staging its tokens overlaps the
+// other CTAs' weight streams).  The expert's
 // activations for a chunk of up to `nx` tokens are staged once per CTA in shared memory,
 // already paired the way the dequantised weights pair them and with their per-group sums.
 // Each warp then streams its own units group by group (16 rows x 128 K-elements per group)
@@ -21,12 +23,12 @@ namespace moe {
 
 enum { kGateUp = 0, kDown = 1 };
 constexpr int kRows = 16;     // weight rows per unit
-constexpr int kWarps = 8;     // warps per CTA, each owning whole units
+constexpr int kWarps = 4;     // warps per CTA, each owning whole units
 constexpr int kThreads = 32 * kWarps;
 constexpr int kDepth = 6;     // group steps in flight per warp (bitplane, NVFP4)
 constexpr int kDepthW4 = 8;   // W4: groups in flight per warp, consumed and refilled two at a time
 constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
-constexpr size_t kSmemTarget = 110 * 1024;  // two CTAs per SM
+constexpr size_t kSmemTarget = 55 * 1024;  // four CTAs per SM
 
 struct FfnArgs {
   const void* act;  // gate/up: x bf16 [T][K]; down: h [P][K] (bf16, or fp16*2^-8 for NVFP4)
@@ -312,7 +314,7 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t
 
 // ---------------------------------------------------------------- kernel
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, 2) k_ffn_gemv(FfnArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int slot = blockIdx.y;
