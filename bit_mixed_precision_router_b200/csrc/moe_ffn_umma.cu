@@ -74,7 +74,8 @@ constexpr int kEpiWarp0 = kDeqWarp0 + 4 * kDeqSets;
 constexpr int kOffB = 0;
 constexpr int kOffW = kOffB + kBStages * kBStageBytes;
 constexpr int kOffPre = kOffW + kWStages * kWStageBytes;  // tile prefix over experts
-constexpr int kOffBar = kOffPre + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
+constexpr int kOffOffs = kOffPre + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;  // routing offsets
+constexpr int kOffBar = kOffOffs + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
 constexpr int kNumBars = 2 * kBStages + 2 * kWStages + 2 * kAStages + 4;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffTmemSlot + 16;
@@ -226,7 +227,8 @@ struct Tile {
   int e, r0, nrows, wt;
 };
 
-MOE_DEVICE Tile tile_of(int item, const int* pre, int E, int wtiles, const int32_t* offsets) {
+// `offsets` is the CTA's shared-memory copy of the routing offsets.
+MOE_DEVICE Tile tile_of(int item, const int* pre, int E, int wtiles, const int* offsets) {
   const int t = item / wtiles;
   Tile tl;
   tl.wt = item - t * wtiles;
@@ -251,6 +253,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
   int* pre = reinterpret_cast<int*>(smem + kOffPre);
+  int* offs = reinterpret_cast<int*>(smem + kOffOffs);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* fullB = bars;
   uint64_t* emptyB = fullB + kBStages;
@@ -265,12 +268,15 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E;
 
+  // ---- the routing offsets into shared memory (every role reads them per tile)
+  for (int i = tid; i <= E; i += blockDim.x) offs[i] = a.offsets[i];
+  __syncthreads();
   // ---- tiles per expert and their prefix (warp 0), barriers (warp 2), tensor memory (warp 1)
   if (warp == 0) {
     const int per = (E + 31) / 32;
     const int b = min(E, lane * per), en = min(E, b + per);
     int sum = 0;
-    for (int e = b; e < en; ++e) sum += (a.offsets[e + 1] - a.offsets[e] + kTN - 1) / kTN;
+    for (int e = b; e < en; ++e) sum += (offs[e + 1] - offs[e] + kTN - 1) / kTN;
     int inc = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     int run = inc - sum;
     for (int e = b; e < en; ++e) {
       pre[e] = run;
-      run += (a.offsets[e + 1] - a.offsets[e] + kTN - 1) / kTN;
+      run += (offs[e + 1] - offs[e] + kTN - 1) / kTN;
     }
     if (lane == 31) pre[E] = inc;
   } else if (tid == 64) {
@@ -317,7 +323,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     int n = 0;  // k-blocks issued
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
+      const Tile tl = tile_of(item, pre, E, a.wtiles, offs);
       int wr0, wr1;  // weight box rows
       if (MODE == kGateUp) {
         wr0 = tl.e * a.n_rows + tl.wt * 64;
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       bool ok = true;
       const uint64_t bdesc0 = sw128_desc(sbase + kOffB);
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
-        const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
+        const Tile tl = tile_of(item, pre, E, a.wtiles, offs);
         const int ab = it & 1;
         if (!mbar_wait(&accEmpty[ab], ((it >> 1) & 1) ^ 1, a.err)) break;
         tc_fence_after();
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int li = n / KB, grp = n - li * KB;
       if (li != s_li) {
         s_li = li;
-        const Tile tl = tile_of(int(blockIdx.x) + li * int(gridDim.x), pre, E, a.wtiles, a.offsets);
+        const Tile tl = tile_of(int(blockIdx.x) + li * int(gridDim.x), pre, E, a.wtiles, offs);
         int r;
         if (MODE == kGateUp) r = (srow < 64) ? tl.wt * 64 + srow : a.I + tl.wt * 64 + (srow - 64);
         else r = tl.wt * kTM + srow;
@@ -494,7 +500,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     int it = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
-      const Tile tl = tile_of(item, pre, E, a.wtiles, a.offsets);
+      const Tile tl = tile_of(item, pre, E, a.wtiles, offs);
       const int ab = it & 1;
       if (!warp_wait(&accFull[ab], (it >> 1) & 1, a.err)) break;
       tc_fence_after();
