@@ -90,9 +90,10 @@ MOE_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: 
 // eight weights.  The activations were staged as fp16 x/16 opposite the first kind and
 // x/256 opposite the second, so each product is (1032 + q) x/16 or (72 + q) x/16 (q = u - 8);
 // the accumulator starts at the staged seed -(1032 sum x/16 + 1152 sum x/256) of the
-// group and ends at sum q x/16, scaled by 16 s into the row's sum.
+// group and ends at sum q x/16, scaled by s into the row's sum (the factor 16 is applied
+// once, in the epilogue).
 template <bool TWO>
-MOE_DEVICE void w4h_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa16, float sb16,
+MOE_DEVICE void w4h_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa, float sb,
                           const float (&S)[2][2], float (&acc)[2][4]) {
   const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
   const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
@@ -120,10 +121,10 @@ MOE_DEVICE void w4h_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa1
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    acc[nt][0] = fmaf(sa16, t[nt][0], acc[nt][0]);
-    acc[nt][1] = fmaf(sa16, t[nt][1], acc[nt][1]);
-    acc[nt][2] = fmaf(sb16, t[nt][2], acc[nt][2]);
-    acc[nt][3] = fmaf(sb16, t[nt][3], acc[nt][3]);
+    acc[nt][0] = fmaf(sa, t[nt][0], acc[nt][0]);
+    acc[nt][1] = fmaf(sa, t[nt][1], acc[nt][1]);
+    acc[nt][2] = fmaf(sb, t[nt][2], acc[nt][2]);
+    acc[nt][3] = fmaf(sb, t[nt][3], acc[nt][3]);
   }
 }
 
@@ -229,10 +230,11 @@ MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* 
                           const float* xsum, int GK, int g, int c, int nvalid, Issue&& issue, float (&acc)[2][4]) {
   constexpr int NT = TWO ? 2 : 1;
   constexpr int D = kDepthW4;
-  const uint8_t* xr[2] = {xbuf + size_t(g) * a.x_stride + c * 16, xbuf + size_t(8 + g) * a.x_stride + c * 16};
-  const bool live[2] = {g < nvalid, 8 + g < nvalid};
-  const float* sr[2][2] = {{xsum + (2 * c) * GK, xsum + (2 * c + 1) * GK},
-                           {xsum + (8 + 2 * c) * GK, xsum + (8 + 2 * c + 1) * GK}};
+  // B column of an absent token: any staged row will do (each output column depends only
+  // on its own B column, and absent columns are never stored)
+  const uint8_t* xr[2] = {xbuf + size_t(min(g, nvalid - 1)) * a.x_stride + c * 16,
+                          xbuf + size_t(min(8 + g, nvalid - 1)) * a.x_stride + c * 16};
+  const float* sr = xsum + 2 * c;  // seeds [G][kMaxTok]: columns 2c, 2c+1 (+8 for the second tile)
   const uint16_t* wsa = wscale + g * GK;
   const uint16_t* wsb = wscale + (g + 8) * GK;
   const uint8_t* wl = wsm + g * 64 + c * 16;
@@ -248,14 +250,14 @@ MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* 
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-          for (int m = 0; m < 4; ++m)
-            xv[nt][m] = live[nt] ? *reinterpret_cast<const uint4*>(xr[nt] + GG * 256 + m * 64) : make_uint4(0, 0, 0, 0);
-          S[nt][0] = sr[nt][0][GG];
-          S[nt][1] = sr[nt][1][GG];
+          for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr[nt] + GG * 256 + m * 64);
+          const float2 s2 = *reinterpret_cast<const float2*>(sr + GG * kMaxTok + 8 * nt);
+          S[nt][0] = s2.x;
+          S[nt][1] = s2.y;
         }
         const uint8_t* wr = wl + (GG & (D - 1)) * 1024;
         w4h_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
-                       16.f * bf16_bits_to_float(wsa[GG]), 16.f * bf16_bits_to_float(wsb[GG]), S, acc);
+                       bf16_bits_to_float(wsa[GG]), bf16_bits_to_float(wsb[GG]), S, acc);
       }
     }
     __syncwarp();  // every lane is done with these slots before they are refilled
@@ -282,17 +284,16 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t
     float X[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      if (nt * 8 + g >= nvalid) {  // B column of an absent token
+      // B column of an absent token: any staged row will do (each output column depends
+      // only on its own B column, and absent columns are never stored)
+      const int row = min(nt * 8 + g, nvalid - 1);
+      const uint8_t* xr = xbuf + size_t(row) * a.x_stride + G * 256 + c * 16;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) xv[nt][m] = make_uint4(0, 0, 0, 0);
-      } else {
-        const uint8_t* xr = xbuf + size_t(nt * 8 + g) * a.x_stride + G * 256 + c * 16;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
-      }
-      if (FMT != MOE_FMT_NVFP4) {  // group sums of C columns 2c, 2c+1 (kMaxTok rows staged)
-        X[nt][0] = xsum[(nt * 8 + 2 * c) * GK + G];
-        X[nt][1] = xsum[(nt * 8 + 2 * c + 1) * GK + G];
+      for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
+      if (FMT != MOE_FMT_NVFP4) {  // group sums of C columns 2c, 2c+1 ([G][kMaxTok] staged)
+        const float2 x2 = *reinterpret_cast<const float2*>(xsum + G * kMaxTok + nt * 8 + 2 * c);
+        X[nt][0] = x2.x;
+        X[nt][1] = x2.y;
       }
     }
     if (FMT == MOE_FMT_BITPLANE8) {
@@ -510,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
       if (FMT != MOE_FMT_NVFP4) {  // group sums: the 4 slices of a group are 4 consecutive lanes
         ssum += __shfl_xor_sync(0xffffffffu, ssum, 1);
         ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
-        if (ok && (sl & 3) == 0) xsum[n * GK + (sl >> 2)] = ssum;
+        if (ok && (sl & 3) == 0) xsum[(sl >> 2) * kMaxTok + n] = ssum;
       }
     }
     if (FMT == MOE_FMT_BITPLANE8)
@@ -549,6 +550,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
     // ---- epilogue: C fragment = rows g / g+8, tokens 2c, 2c+1 of each n8 tile
     float post = 1.f;
     if (FMT == MOE_FMT_NVFP4) post = a.gscale[e] * 256.f;
+    if (FMT == MOE_FMT_W4G128) post = 16.f;  // the activations were staged as x/16
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
