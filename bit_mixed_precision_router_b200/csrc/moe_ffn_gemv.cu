@@ -26,7 +26,7 @@ constexpr int kRows = 16;     // weight rows per unit
 constexpr int kWarps = 4;     // warps per CTA, each owning whole units
 constexpr int kThreads = 32 * kWarps;
 constexpr int kDepth = 6;     // group steps in flight per warp (bitplane, NVFP4)
-constexpr int kDepthW4 = 8;   // W4: groups in flight per warp, consumed and refilled two at a time
+constexpr int kDepthW4 = 6;   // W4: groups in flight per warp, consumed and refilled two at a time
 constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
 constexpr size_t kSmemTarget = 55 * 1024;  // four CTAs per SM
 
@@ -255,7 +255,7 @@ MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* 
           S[nt][0] = s2.x;
           S[nt][1] = s2.y;
         }
-        const uint8_t* wr = wl + (GG & (D - 1)) * 1024;
+        const uint8_t* wr = wl + (GG % D) * 1024;
         w4h_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
                        bf16_bits_to_float(wsa[GG]), bf16_bits_to_float(wsb[GG]), S, acc);
       }
