@@ -214,14 +214,21 @@ size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64
  * For sorted row r of expert e holding pair p = t*k + j:
  *   g = x[t] . deq(W_gate_e)^T, u = x[t] . deq(W_up_e)^T  (fp32 accumulation),
  *   h = bf16(silu(g) * u),  y_rows[r] = bf16(h . deq(W2_e)^T).
- * Dequantisation happens in registers; for BITPLANE8 expert e is read at bits[p]
- * planes for pair p (planes 0..bits[p]-1, floor and compensation as above).
+ * Two execution paths, chosen on the host from the shape alone (nothing is read back
+ * from the device): with T*k >= 32*E and W4G128 or NVFP4 weights, a tensor-core GEMM
+ * (weights dequantised into tensor memory once per tile of up to 192 routed rows,
+ * bf16 operands for W4, fp16 for NVFP4); otherwise a weight-streaming GEMV
+ * (dequantisation in registers, weights read once per pass of up to 16 rows).  For
+ * BITPLANE8 expert e is read at bits[p] planes for pair p (planes 0..bits[p]-1, floor
+ * and compensation as above); expert e's weights are fetched to max_p bits[p].
  *   x bf16 [T][H];  routing: as written by moe_route_topk;  bits uint8 [T*k]
  *   (BITPLANE8 only, values 1..8, else may be NULL);  y_rows bf16 [T*k][H].
  * Requires H % 256 == 0, I % 128 == 0, the limits of moe_route_topk, and workspace
- * >= moe_ffn_workspace_bytes(...).  Not bit-exact: fp32 accumulation order and the
- * bf16 rounding of h differ from an fp64 reference (ExactMoE: the low-bit layer is
- * not numerically identical to BF16). */
+ * >= moe_ffn_workspace_bytes(...) (scratch: h, and for the GEMM path the token rows
+ * gathered into routed order; contents need not be initialised).  Not bit-exact: fp32
+ * accumulation order, the rounding of h (and, on the GEMM path, of each dequantised
+ * W4 weight to bf16) differ from an fp64 reference (ExactMoE: the low-bit layer is
+ * not numerically identical to BF16); the FFN tolerance covers both paths. */
 moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
                              const moe_experts_t* experts, const uint8_t* bits,
                              int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,

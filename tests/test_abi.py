@@ -95,6 +95,10 @@ def test_ffn_and_combine_validation(lib):
     ex.fmt = 7
     assert call(4, 2048, 1024, 64, 8) == INVALID
     assert lib.moe_ffn_workspace_bytes(16, 2048, 1024, 64, 8, 0) >= 16 * 8 * 1024 * 2
+    # tensor-core path (T*k >= 32*E): h plus the token rows gathered into routed order
+    P = 2048 * 8
+    for fmt in (0, 2):
+        assert lib.moe_ffn_workspace_bytes(2048, 2048, 768, 128, 8, fmt) >= P * 768 * 2 + P * 2048 * 2
     c = lambda T, H, k, res=None: lib.moe_combine(A, ctypes.byref(r), res, T, H, k, A, None)
     assert c(4, 2044, 8) == SHAPE
     assert c(4, 2048, 0) == INVALID
