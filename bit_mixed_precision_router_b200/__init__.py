@@ -59,6 +59,11 @@ _SIGS = {
                                ctypes.c_int),
     "moe_select_bits": ([_vp, _i64, _i64, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_uint8), _vp,
                          _vp], ctypes.c_int),
+    "moe_bitplane_distortion": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
+    "moe_activation_moments": ([_vp, _i64, _i64, _vp, _vp], ctypes.c_int),
+    "moe_allocate_bits": ([_vp, _vp, _vp, _i64, _i64, ctypes.POINTER(ctypes.c_uint8), _i64, _d, _vp, _vp, _vp],
+                          ctypes.c_int),
+    "moe_expand_bits": ([_vp, _vp, _i64, _i64, _vp, _vp], ctypes.c_int),
     "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
     "moe_grouped_ffn": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
                          _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
@@ -220,6 +225,47 @@ def moe_select_bits(topk_w: torch.Tensor, k: int, thresholds=(0.05, 0.15, 0.30),
     thr = (ctypes.c_float * 3)(*thresholds)
     ch = (ctypes.c_uint8 * 4)(*choices)
     _call("moe_select_bits", _p(topk_w), T, k, thr, ch, _p(bits), _stream(stream))
+    return bits
+
+
+# ---------------------------------------------------------------- budgeted bit allocation
+def moe_bitplane_distortion(planes: torch.Tensor, scales: torch.Tensor, delta: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
+    """delta fp64 [E][8][K] of a bitplane matrix planes [E][8][N][K/32], scales [E][N][K/128]."""
+    E, _, N, K32 = planes.shape
+    K = K32 * 32
+    delta = torch.empty((E, 8, K), dtype=torch.float64, device=planes.device) if delta is None else delta
+    _call("moe_bitplane_distortion", _p(planes), _p(_bits(scales)), E, N, K, _p(delta), _stream(stream))
+    return delta
+
+
+def moe_activation_moments(x: torch.Tensor, m: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """m fp64 [H]: mean over the T tokens of x [T][H] (bf16) squared."""
+    T, H = x.shape
+    m = torch.empty(H, dtype=torch.float64, device=x.device) if m is None else m
+    _call("moe_activation_moments", _p(_bits(x)), T, H, _p(m), _stream(stream))
+    return m
+
+
+def moe_allocate_bits(delta: torch.Tensor, m: torch.Tensor, expert_offsets: torch.Tensor, budget: float,
+                      choices=(2, 3, 4, 8), bits_e: torch.Tensor | None = None, lam: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """uint8 [E] per-expert widths under a read budget (bits per weight); the final
+    multiplier is written to ``lam`` (fp64 scalar tensor) when given."""
+    E, _, K = delta.shape
+    bits_e = torch.empty(E, dtype=torch.uint8, device=delta.device) if bits_e is None else bits_e
+    ch = (ctypes.c_uint8 * len(choices))(*choices)
+    _call("moe_allocate_bits", _p(delta), _p(m), _p(expert_offsets), E, K, ch, len(choices), float(budget),
+          _p(bits_e), _p(lam), _stream(stream))
+    return bits_e
+
+
+def moe_expand_bits(topk_ids: torch.Tensor, bits_e: torch.Tensor, k: int, bits: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Per-pair widths bits[p] = bits_e[topk_ids[p]] for moe_grouped_ffn."""
+    n = topk_ids.numel()
+    bits = torch.empty(max(n, 1), dtype=torch.uint8, device=topk_ids.device) if bits is None else bits
+    _call("moe_expand_bits", _p(topk_ids), _p(bits_e), n // k, k, _p(bits), _stream(stream))
     return bits
 
 

@@ -129,6 +129,50 @@ moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const f
                                      as_stream(stream)));
 }
 
+moe_status_t moe_bitplane_distortion(const uint32_t* planes, const uint16_t* scales, int64_t E, int64_t N,
+                                     int64_t K, double* delta, moe_stream_t stream) {
+  if (!planes || !scales || !delta) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || N < 1 || K < 1) return MOE_ERR_INVALID_ARG;
+  if (K % 128 != 0 || E > INT_MAX || N > INT_MAX || K > INT_MAX || E * K > INT_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(planes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(delta) & 7u)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_bitplane_distortion(planes, scales, int(E), int(N), int(K), delta, as_stream(stream)));
+}
+
+moe_status_t moe_activation_moments(const uint16_t* x, int64_t T, int64_t H, double* m, moe_stream_t stream) {
+  if (!x || !m) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1) return MOE_ERR_INVALID_ARG;
+  if (T > INT_MAX || H > INT_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (reinterpret_cast<uintptr_t>(m) & 7u)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_act_moments(x, int(T), int(H), m, as_stream(stream)));
+}
+
+moe_status_t moe_allocate_bits(const double* delta, const double* m, const int32_t* expert_offsets, int64_t E,
+                               int64_t K, const uint8_t* choices, int64_t nchoices, double budget,
+                               uint8_t* bits_e, double* lambda, moe_stream_t stream) {
+  if (!delta || !m || !expert_offsets || !choices || !bits_e) return MOE_ERR_INVALID_ARG;
+  if (nchoices < 1 || nchoices > 8 || !(budget >= 0.0) || budget > 1e300) return MOE_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < nchoices; ++i) {
+    if (choices[i] < 1 || choices[i] > 8) return MOE_ERR_INVALID_ARG;
+    for (int64_t j = 0; j < i; ++j)
+      if (choices[j] == choices[i]) return MOE_ERR_INVALID_ARG;
+  }
+  if (E < 1 || E > MOE_MAX_EXPERTS || K < 1 || K > INT_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(delta) & 7u) || (reinterpret_cast<uintptr_t>(m) & 7u) ||
+      (reinterpret_cast<uintptr_t>(expert_offsets) & 3u) || (lambda && (reinterpret_cast<uintptr_t>(lambda) & 7u)))
+    return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_allocate_bits(delta, m, expert_offsets, int(E), int(K), choices, int(nchoices),
+                                             budget, bits_e, lambda, as_stream(stream)));
+}
+
+moe_status_t moe_expand_bits(const int32_t* topk_ids, const uint8_t* bits_e, int64_t T, int64_t k,
+                             uint8_t* bits, moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!topk_ids || !bits_e || !bits) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(topk_ids) & 3u) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_expand_bits(topk_ids, bits_e, T * k, bits, as_stream(stream)));
+}
+
 moe_status_t moe_select_bits(const float* topk_w, int64_t T, int64_t k, const float thresholds[3],
                              const uint8_t choices[4], uint8_t* bits, moe_stream_t stream) {
   if (!topk_w || !thresholds || !choices || !bits) return MOE_ERR_INVALID_ARG;

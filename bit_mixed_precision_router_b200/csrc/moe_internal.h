@@ -38,6 +38,16 @@ size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
 cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
                                     int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st);
 
+// Budgeted per-expert bit allocation (moe_alloc.cu).
+cudaError_t launch_bitplane_distortion(const uint32_t* planes, const uint16_t* scales, int E, int N, int K,
+                                       double* delta, cudaStream_t st);
+cudaError_t launch_act_moments(const uint16_t* x, int T, int H, double* m, cudaStream_t st);
+cudaError_t launch_allocate_bits(const double* delta, const double* m, const int32_t* offsets, int E, int K,
+                                 const uint8_t* choices, int nchoices, double budget, uint8_t* bits_e,
+                                 double* lam_out, cudaStream_t st);
+cudaError_t launch_expand_bits(const int32_t* ids, const uint8_t* bits_e, int64_t n, uint8_t* bits,
+                               cudaStream_t st);
+
 cudaError_t launch_combine(const uint16_t* y_rows, const moe_routing_t& r, const uint16_t* residual, int T,
                            int H, int k, uint16_t* out, cudaStream_t st);
 

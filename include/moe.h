@@ -193,6 +193,50 @@ moe_status_t moe_route_topk_noalloc(const uint16_t* x, const uint16_t* w_router,
                                     int64_t T, int64_t H, int64_t E, int64_t k,
                                     const moe_routing_t* out, moe_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Budgeted bit allocation for bitplane experts (replaces the fixed thresholds of
+ * moe_select_bits with a per-expert choice under a read budget)
+ * ------------------------------------------------------------------------ */
+
+/* Offline distortion table [DuoRate: a distortion tensor baked offline].  For expert
+ * e, prefix length b = 1..8 and input channel k:
+ *   delta[e][b-1][k] = sum_{n<N} (s[e][n][k/128] * (u'_b[e][n][k] - u[e][n][k]))^2,
+ * u the stored 8-bit code, u'_b its b-bit floor-and-compensation prefix (0 for b = 8),
+ * fp64, rows n in order.  Pass the gate/up matrix (K = H: the matrix that reads x).
+ *   planes uint32 [E][8][N][K/32] and scales bf16 [E][N][K/128] as written by
+ *   moe_pack_bitplanes;  delta fp64 [E][8][K] (caller-allocated).
+ * Requires E, N >= 1, K % 128 == 0. */
+moe_status_t moe_bitplane_distortion(const uint32_t* planes, const uint16_t* scales, int64_t E, int64_t N,
+                                     int64_t K, double* delta, moe_stream_t stream);
+
+/* Activation second moments of a workload's tokens [DuoRate: online profiling of a
+ * workload's prefill, without labels]: m[k] = (1/T) sum_t x[t][k]^2, fp64, tokens in
+ * order.   x bf16 [T][H];  m fp64 [H].  Requires T, H >= 1. */
+moe_status_t moe_activation_moments(const uint16_t* x, int64_t T, int64_t H, double* m, moe_stream_t stream);
+
+/* Per-expert bit-widths under a read budget [DuoRate: a Lagrangian rate-distortion
+ * allocation solved with one dot product per expert and a bisection to the read
+ * budget; the routing frequency cancels from every per-expert decision].
+ *   D[e][c] = sum_k m[k] * delta[e][choices[c]-1][k]  (one warp per dot product);
+ *   at multiplier lam each expert takes argmin_c D[e][c] + lam * choices[c], ties to the
+ *   larger width; 100 bisection steps on lam find the smallest lam whose read rate is
+ *   within the budget -- the exact integer sum_e n_e * b_e (n_e pairs routed to e, from
+ *   expert_offsets) against the fp64 product budget * sum_e n_e -- and bits_e receives
+ *   the widths at the upper end of the final interval.  Experts with no pairs, and all
+ *   experts when even the smallest width exceeds the budget, get the smallest choice.
+ *   delta fp64 [E][8][K];  m fp64 [K];  expert_offsets int32 [E+1] (moe_route_topk);
+ *   choices: HOST array of nchoices distinct widths in 1..8, 1 <= nchoices <= 8;
+ *   budget: bits per weight, finite, >= 0;  bits_e uint8 [E];  lambda: fp64 device
+ *   scalar that receives the final multiplier, or NULL.  One CTA; E <= MOE_MAX_EXPERTS. */
+moe_status_t moe_allocate_bits(const double* delta, const double* m, const int32_t* expert_offsets, int64_t E,
+                               int64_t K, const uint8_t* choices, int64_t nchoices, double budget,
+                               uint8_t* bits_e, double* lambda, moe_stream_t stream);
+
+/* Per-pair bit-widths from per-expert ones: bits[p] = bits_e[topk_ids[p]], p < T*k
+ * (the bits array moe_grouped_ffn takes for BITPLANE8). */
+moe_status_t moe_expand_bits(const int32_t* topk_ids, const uint8_t* bits_e, int64_t T, int64_t k,
+                             uint8_t* bits, moe_stream_t stream);
+
 /* Per-pair bit-width from the routing weight [MatMoE: precision per expert from
  * routing scores; PagedMoE: prefix length from current routing weights].
  * bits[p] = choices[0] if w < thresholds[0], choices[1] if w < thresholds[1],

@@ -116,3 +116,45 @@ def test_select_bits_validation(lib):
     assert lib.moe_select_bits(A, 0, 8, thr, ch, A, None) == OK
     assert lib.moe_synth_normal_bf16(None, 4, 0, 1, 1.0, None) == INVALID
     assert lib.moe_synth_normal_bf16(A, 0, 0, 1, 1.0, None) == OK
+
+
+def test_allocation_validation(lib):
+    nan, inf = float("nan"), float("inf")
+    d = lambda E, N, K, planes=A, delta=A: lib.moe_bitplane_distortion(planes, A, E, N, K, delta, None)
+    assert d(4, 8, 2048, planes=None) == INVALID
+    assert d(0, 8, 2048) == INVALID
+    assert d(4, 0, 2048) == INVALID
+    assert d(4, 8, 2000) == SHAPE
+    assert d(4, 8, 2048, planes=A + 4) == MISALIGNED
+    assert d(4, 8, 2048, delta=A + 4) == MISALIGNED
+    m = lambda T, H, x=A, out=A: lib.moe_activation_moments(x, T, H, out, None)
+    assert m(0, 2048) == INVALID
+    assert m(4, 0) == INVALID
+    assert m(4, 2048, x=None) == INVALID
+    assert m(4, 2048, x=A + 1) == MISALIGNED
+    assert m(4, 2048, out=A + 4) == MISALIGNED
+
+    def alloc(E, K, choices, budget, offs=A, lam=None):
+        ch = (ctypes.c_uint8 * max(len(choices), 1))(*choices)
+        return lib.moe_allocate_bits(A, A, offs, E, K, ch, len(choices), budget, A, lam, None)
+    assert alloc(64, 2048, (2, 3, 4, 8), nan) == INVALID
+    assert alloc(64, 2048, (2, 3, 4, 8), -0.5) == INVALID
+    assert alloc(64, 2048, (2, 3, 4, 8), inf) == INVALID
+    assert alloc(64, 2048, (), 4.0) == INVALID
+    assert alloc(64, 2048, (1, 2, 3, 4, 5, 6, 7, 8, 8), 4.0) == INVALID
+    assert alloc(64, 2048, (2, 3, 3), 4.0) == INVALID
+    assert alloc(64, 2048, (0, 3), 4.0) == INVALID
+    assert alloc(64, 2048, (2, 9), 4.0) == INVALID
+    assert alloc(0, 2048, (2, 8), 4.0) == SHAPE
+    assert alloc(1025, 2048, (2, 8), 4.0) == SHAPE
+    assert alloc(64, 0, (2, 8), 4.0) == SHAPE
+    assert alloc(64, 2048, (2, 8), 4.0, offs=A + 2) == MISALIGNED
+    assert alloc(64, 2048, (2, 8), 4.0, lam=A + 4) == MISALIGNED
+    assert lib.moe_allocate_bits(None, A, A, 64, 2048, (ctypes.c_uint8 * 2)(2, 8), 2, 4.0, A, None, None) == INVALID
+    e = lambda T, k, ids=A: lib.moe_expand_bits(ids, A, T, k, A, None)
+    assert e(-1, 8) == INVALID
+    assert e(4, 0, ) == INVALID
+    assert e(4, 33) == INVALID
+    assert e(4, 8, ids=None) == INVALID
+    assert e(4, 8, ids=A + 2) == MISALIGNED
+    assert e(0, 8, ids=None) == OK
