@@ -11,11 +11,15 @@ as one CUDA graph.  `value` = tokens per second through the 16-layer stack
 (a token counts once per step), whole job over all ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl reference]
-                    [--workload decode|prefill-h2048-e128|prefill-h7168-e256]
+                    [--workload decode|prefill-h2048-e128|prefill-h7168-e256|prefill-h7168-e256-nvfp4|
+                                bitplane-h2048-e64]
 
 The prefill workloads (not the default) time one MoE FFN layer on a large batch
 of fresh tokens per step -- the tensor-core grouped GEMM path -- and report its
-roofline against the measured bf16 tensor peak.
+roofline against the measured bf16 tensor peak.  The bitplane workload times one
+layer of 8-bitplane experts on 64 tokens per step, each expert read at the width a
+budgeted allocation gave it (allocated once, before timing, from a profiling batch;
+the allocation kernels' times are reported in the config), against the HBM peak.
 
 Under torchrun each rank runs its own replica on its own seeded batches (the
 layer shards by token, no data-path collective): weak scaling, time = max over
@@ -56,7 +60,16 @@ PREFILL = {
                                      desc="one MoE FFN layer, H7168 I2048 E256 top-8, NVFP4 experts (E2M1, E4M3 "
                                           "per 16, fp32 per tensor), U(-0.02, 0.02) bf16 router, 4096 fresh "
                                           "tokens per step"),
+    "bitplane-h2048-e64": dict(T=64, H=2048, I=1024, E=64, k=8, router="normal", zipf=False, seed=0x5EED0004,
+                               fmt="bitplane", budget=3.0, choices=(2, 3, 4, 8), profile_tokens=2048,
+                               desc="one MoE FFN layer, H2048 I1024 E64 top-8, 8-bitplane experts read at "
+                                    "per-expert widths from a budgeted allocation (3.0 bits per weight of "
+                                    "routing-weighted reads over {2,3,4,8}, profiled on 2048 tokens), bf16 "
+                                    "router, 64 fresh tokens per step"),
 }
+# bitplane experts: bytes of one plane of one expert's w13 + w2, and of their bf16 scales
+BP_PLANE_BYTES = (2 * I * H + H * I) // 8
+BP_SCALE_BYTES = (2 * I * (H // 128) + H * (I // 128)) * 2
 
 
 def parse_args(argv=None):
@@ -73,7 +86,7 @@ def parse_args(argv=None):
                     help="layers in the stack (16 is the benchmark workload; fewer only for profiling)")
     args = ap.parse_args(argv)
     if args.steps is None:
-        args.steps = 512 if args.workload == "decode" else 20
+        args.steps = 512 if args.workload in ("decode", "bitplane-h2048-e64") else 20
     return args
 
 
@@ -174,10 +187,10 @@ def measured_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def committed_traffic():
-    """DRAM bytes per moe_grouped_ffn call (gate/up + down launches) from the committed
+def committed_traffic(name: str = "traffic.json"):
+    """DRAM bytes of moe_grouped_ffn calls (gate/up + down launches) from the committed
     ncu summary, with the kernel source hash it was taken on (None if stale/absent)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", name)
     try:
         d = json.load(open(path))
     except (OSError, ValueError):
@@ -397,10 +410,13 @@ class PrefillLayer:
         seed = cfg["seed"]
         i32, bf = dict(dtype=torch.int32, device=device), dict(dtype=torch.bfloat16, device=device)
         u8, f32 = dict(dtype=torch.uint8, device=device), dict(dtype=torch.float32, device=device)
-        self.fmt = moe.FMT_NVFP4 if cfg.get("fmt") == "nvfp4" else moe.FMT_W4G128
+        self.fmt = {"nvfp4": moe.FMT_NVFP4, "bitplane": moe.FMT_BITPLANE8}.get(cfg.get("fmt"), moe.FMT_W4G128)
         if self.fmt == moe.FMT_NVFP4:
             mk = lambda n, kk: (torch.empty((Ee, n, kk // 2), **u8), torch.empty((Ee, n, kk // 16), **u8),
                                 torch.empty((Ee,), **f32))
+        elif self.fmt == moe.FMT_BITPLANE8:
+            mk = lambda n, kk: (torch.empty((Ee, 8, n, kk // 32), **i32), torch.empty((Ee, n, kk // 128), **bf),
+                                None)
         else:
             mk = lambda n, kk: (torch.empty((Ee, n, kk // 8), **i32), torch.empty((Ee, n, kk // 128), **bf), None)
         w13, w2 = mk(2 * Ii, Hh), mk(Hh, Ii)
@@ -412,6 +428,8 @@ class PrefillLayer:
                 moe.moe_synth_normal_bf16(t, seed + tag, 0.02, start=e0 * n * kk)
                 if self.fmt == moe.FMT_NVFP4:
                     moe.moe_quantize_nvfp4(t, st[0][e0:e0 + ne], st[1][e0:e0 + ne], st[2][e0:e0 + ne])
+                elif self.fmt == moe.FMT_BITPLANE8:
+                    moe.moe_pack_bitplanes(t, st[0][e0:e0 + ne], st[1][e0:e0 + ne])
                 else:
                     moe.moe_quantize_w4g128(t, st[0][e0:e0 + ne], st[1][e0:e0 + ne])
         del tmp
@@ -431,19 +449,74 @@ class PrefillLayer:
         self.x = torch.empty((T, Hh), **bf)
         self.out = torch.empty((T, Hh), **bf)
         self.ffn_events = None
+        self.bits_e = self.bits = None
+        self.copies = [self.experts]
+        if self.fmt == moe.FMT_BITPLANE8:
+            self.bits = torch.empty((T * k,), **u8)
+            # a step reads only ~b_e planes of each expert (about 160 MB, near the 126 MB L2):
+            # steps rotate over 4 device copies of the same weights so no step finds the
+            # previous step's planes in L2
+            for _ in range(3):
+                self.copies.append(moe.Experts(self.fmt, w13[0].clone(), w13[1].clone(), w2[0].clone(),
+                                               w2[1].clone(), None, None))
 
-    def step(self):
+    def allocate_widths(self, torch, device, seed):
+        """Per-expert widths for the bitplane experts under the read budget: the distortion
+        tensor of the gate/up matrices (offline), the activation moments of a profiling
+        batch of the workload, the routing counts of that batch, then the allocation.
+        Each of the three kernels is timed with CUDA events (median of 5)."""
+        import synth
+        moe, c = self.moe, self.cfg
+        xp = torch.empty((c["profile_tokens"], c["H"]), dtype=torch.bfloat16, device=device)
+        moe.moe_synth_normal_bf16(xp, seed + synth.SEED_X + 0x51, 1.0)
+        rp = moe.moe_route_topk(xp, self.wr, self.bias, c["k"])
+        delta = torch.empty((c["E"], 8, c["H"]), dtype=torch.float64, device=device)
+        m = torch.empty((c["H"],), dtype=torch.float64, device=device)
+        lam = torch.zeros((), dtype=torch.float64, device=device)
+        self.bits_e = torch.empty((c["E"],), dtype=torch.uint8, device=device)
+        times = {"distortion": [], "moments": [], "allocate": []}
+        for _ in range(5):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record()
+            moe.moe_bitplane_distortion(self.experts.w13, self.experts.w13_scale, delta=delta)
+            ev[1].record()
+            moe.moe_activation_moments(xp, m=m)
+            ev[2].record()
+            moe.moe_allocate_bits(delta, m, rp.expert_offsets, c["budget"], choices=c["choices"],
+                                  bits_e=self.bits_e, lam=lam)
+            ev[3].record()
+            torch.cuda.synchronize()
+            for i, key in enumerate(times):
+                times[key].append(ev[i].elapsed_time(ev[i + 1]) * 1e3)
+        moe.moe_check_device_errors()
+        counts = torch.diff(rp.expert_offsets.to(torch.int64)).cpu()
+        be = self.bits_e.cpu().to(torch.int64)
+        hist = {str(b): int((be == b).sum()) for b in c["choices"]}
+        return {"budget_bits_per_weight": c["budget"], "choices": list(c["choices"]),
+                "profile_tokens": c["profile_tokens"], "widths_histogram": hist,
+                "profile_read_rate": round(float((counts * be).sum()) / float(counts.sum()), 4),
+                "resident_rate_mean_width": round(float(be.double().mean()), 4), "lambda": lam.item(),
+                "kernel_us": {key: round(statistics.median(v), 1) for key, v in times.items()}}
+
+    def step(self, copy: int = 0):
         moe, c = self.moe, self.cfg
         moe.moe_route_topk(self.x, self.wr, self.bias, c["k"], out=self.routing, workspace=self.route_ws)
+        if self.bits is not None:
+            moe.moe_expand_bits(self.routing.topk_ids, self.bits_e, c["k"], bits=self.bits)
         if self.ffn_events is not None:
             self.ffn_events[0].record()
-        moe.moe_grouped_ffn(self.x, self.routing, self.experts, c["I"], c["E"], c["k"], y_rows=self.y_rows,
-                            workspace=self.ffn_ws)
+        moe.moe_grouped_ffn(self.x, self.routing, self.copies[copy], c["I"], c["E"], c["k"], y_rows=self.y_rows,
+                            workspace=self.ffn_ws, bits=self.bits)
         if self.ffn_events is not None:
             self.ffn_events[1].record()
         moe.moe_combine(self.y_rows, self.routing, c["T"], c["k"], residual=self.x, out=self.out)
 
-    kernels_per_step = 7  # router logits, top-k, permutation, row gather, gate/up GEMM, down GEMM, combine
+    @property
+    def kernels_per_step(self):
+        # router logits, top-k, permutation (the one-launch router only takes <= 16 tokens of
+        # <= 64 KiB), then the row gather + gate/up + down of the tensor-core path, or
+        # (bitplanes) the width expansion + gate/up + down GEMV, then the combine
+        return 3 + 3 + 1
 
 
 def run_prefill(args, rank, world, local):
@@ -458,6 +531,8 @@ def run_prefill(args, rank, world, local):
     T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
     K, W = args.steps, max(args.warmup, 3)
     layer = PrefillLayer(moe, torch, device, cfg)
+    allocation = layer.allocate_widths(torch, device, rank_seed(cfg["seed"], rank)) \
+        if layer.fmt == moe.FMT_BITPLANE8 else None
     inputs = torch.empty((W + K, T, Hh), dtype=torch.bfloat16, device=device)
     moe.moe_synth_normal_bf16(inputs, rank_seed(cfg["seed"], rank) + synth.SEED_X, 1.0)
     torch.cuda.synchronize()
@@ -465,16 +540,18 @@ def run_prefill(args, rank, world, local):
     layer.step()  # eager first call: device symbols and kernel attributes before capture
     torch.cuda.synchronize()
     moe.moe_check_device_errors()
-    graph = torch.cuda.CUDAGraph()
+    nc = len(layer.copies)
+    graphs = [torch.cuda.CUDAGraph() for _ in range(nc)]
     cap = torch.cuda.Stream(device)
     cap.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap):
-        with torch.cuda.graph(graph, stream=cap):
-            layer.step()
+        for c_, graph in enumerate(graphs):
+            with torch.cuda.graph(graph, stream=cap):
+                layer.step(c_)
     torch.cuda.current_stream().wait_stream(cap)
     for s in range(W):
         layer.x.copy_(inputs[s])
-        graph.replay()
+        graphs[s % nc].replay()
     torch.cuda.synchronize()
     barrier(world)
     clocks = ClockSampler(local)
@@ -484,7 +561,7 @@ def run_prefill(args, rank, world, local):
     ev0.record()
     for s in range(W, W + K):
         layer.x.copy_(inputs[s])
-        graph.replay()
+        graphs[s % nc].replay()
     ev1.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -504,7 +581,7 @@ def run_prefill(args, rank, world, local):
         t0.record()
         for s in range(K):
             layer.x.copy_(host_in[s], non_blocking=True)
-            graph.replay()
+            graphs[s % nc].replay()
             host_out[s].copy_(layer.out, non_blocking=True)
         t1.record()
         torch.cuda.synchronize()
@@ -517,26 +594,44 @@ def run_prefill(args, rank, world, local):
     # of moe_grouped_ffn), CUDA events recorded on its stream inside a graph
     layer.ffn_events = (torch.cuda.Event(enable_timing=True, external=True),
                         torch.cuda.Event(enable_timing=True, external=True))
-    g2 = torch.cuda.CUDAGraph()
+    g2s = [torch.cuda.CUDAGraph() for _ in range(nc)]
     with torch.cuda.stream(cap):
-        with torch.cuda.graph(g2, stream=cap):
-            layer.step()
+        for c_, g2 in enumerate(g2s):
+            with torch.cuda.graph(g2, stream=cap):
+                layer.step(c_)
     torch.cuda.current_stream().wait_stream(cap)
-    ffn_ms = []
+    ffn_ms, ffn_bytes = [], []
+    bits_e = layer.bits_e.cpu().to(torch.int64) if layer.bits_e is not None else None
     for s in range(W, W + min(K, 10)):
         layer.x.copy_(inputs[s])
-        g2.replay()
+        g2s[s % nc].replay()
         torch.cuda.synchronize()
         ffn_ms.append(layer.ffn_events[0].elapsed_time(layer.ffn_events[1]))
+        if bits_e is not None:
+            # the weight stream of this step: each routed expert's prefix of b_e planes, once
+            routed = torch.diff(layer.routing.expert_offsets.to(torch.int64)).cpu() > 0
+            ffn_bytes.append(int((bits_e[routed] * BP_PLANE_BYTES + BP_SCALE_BYTES).sum()))
     layer.ffn_events = None
     hbm, bf16_peak, peak_kind = measured_peaks()
-    flops = 2.0 * T * k * 3 * Hh * Ii
     avg_s = statistics.mean(ffn_ms) / 1e3
-    achieved = flops / avg_s / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
-                "frac": round(achieved / bf16_peak, 4), "peak_kind": peak_kind + " bf16 burst", "traffic": None,
-                "kernel": "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
-                "algorithmic_flops_per_call": flops, "avg_call_us": round(avg_s * 1e6, 1)}
+    if bits_e is not None:
+        achieved = sum(ffn_bytes) / (sum(ffn_ms) / 1e3) / 1e9
+        tr = committed_traffic("traffic_bitplane.json")
+        # DRAM bytes of one captured call (all 64 experts at 3 planes, as this workload allocates)
+        traffic = tr["dram_bytes_per_call"] if tr else None
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4), "peak_kind": peak_kind + " HBM copy", "traffic": traffic,
+                    "kernel": "k_ffn_gemv<bitplane> gate/up + down (one moe_grouped_ffn call)",
+                    "algorithmic_bytes_per_call": round(statistics.mean(ffn_bytes)),
+                    "avg_call_us": round(avg_s * 1e6, 1)}
+    else:
+        flops = 2.0 * T * k * 3 * Hh * Ii
+        achieved = flops / avg_s / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / bf16_peak, 4), "peak_kind": peak_kind + " bf16 burst",
+                    "traffic": None,
+                    "kernel": "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
+                    "algorithmic_flops_per_call": flops, "avg_call_us": round(avg_s * 1e6, 1)}
     result = None
     if rank == 0:
         result = {
@@ -544,17 +639,22 @@ def run_prefill(args, rank, world, local):
             "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16" if cfg.get("fmt") == "nvfp4" else "bf16",
             "data": "synthetic (seeded Irwin-Hall N(0,1) activations, N(0,0.02) bf16 weights quantised to "
-                    + ("NVFP4" if cfg.get("fmt") == "nvfp4" else "W4A16 g128") + ")",
+                    + {"nvfp4": "NVFP4", "bitplane": "8 bitplanes"}.get(cfg.get("fmt"), "W4A16 g128") + ")",
             "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,
                        "top_k": k, "parallelism": f"dp{world} (independent replicas)",
-                       "l2": "no flush: each step reads more than %.1f GB of expert weights, > 126 MB L2"
-                             % (Ee * 3 * Hh * Ii / 2 / 1e9)},
-            "gpu_launches": PrefillLayer.kernels_per_step * K,
+                       "l2": ("no flush: each step reads more than %.1f GB of expert weights, > 126 MB L2"
+                              % (Ee * 3 * Hh * Ii / 2 / 1e9)) if allocation is None else
+                             ("no flush: each step reads about %.0f MB of expert planes and scales, and "
+                              "steps rotate over 4 device copies of the weights (> 126 MB L2 between "
+                              "reuses)" % (statistics.mean(ffn_bytes) / 1e6))},
+            "gpu_launches": layer.kernels_per_step * K,
             "clocks": clk, "roofline": roofline, "e2e": e2e,
         }
+        if allocation is not None:
+            result["config"]["allocation"] = allocation
     if world > 1:
         import torch.distributed as dist
-        del graph, g2
+        del graphs, g2s
         dist.destroy_process_group()
     return result
 
@@ -566,11 +666,13 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
     import numpy as np
 
     import synth
-    from oracle.ffn import FMT_NVFP4, FMT_W4G128, Experts, moe_layer
-    from oracle.quant import quantize_nvfp4, quantize_w4g128
+    from oracle.alloc import expand_bits
+    from oracle.ffn import FMT_BITPLANE8, FMT_NVFP4, FMT_W4G128, Experts, combine, grouped_ffn, moe_layer, route
+    from oracle.quant import pack_bitplanes, quantize_nvfp4, quantize_w4g128
     from oracle.routing import router_logits, topk_softmax
     T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
     nvfp4 = cfg.get("fmt") == "nvfp4"
+    bitplane = cfg.get("fmt") == "bitplane"
     x = synth.normal_bf16(seed + synth.SEED_X, tokens * Hh, 1.0).reshape(tokens, Hh)
     if cfg["router"] == "uniform":
         wr = synth.uniform_bf16(cfg["seed"] + synth.SEED_WR, Ee * Hh, -0.02, 0.02).reshape(Ee, Hh)
@@ -582,6 +684,9 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
         w13q, w13s = np.zeros((Ee, 2 * Ii, Hh // 2), np.uint8), np.zeros((Ee, 2 * Ii, Hh // 16), np.uint8)
         w2q, w2s = np.zeros((Ee, Hh, Ii // 2), np.uint8), np.zeros((Ee, Hh, Ii // 16), np.uint8)
         w13g, w2g = np.zeros(Ee, np.float32), np.zeros(Ee, np.float32)
+    elif bitplane:
+        w13q, w13s = np.zeros((Ee, 8, 2 * Ii, Hh // 32), np.uint32), np.zeros((Ee, 2 * Ii, Hh // 128), np.uint16)
+        w2q, w2s = np.zeros((Ee, 8, Hh, Ii // 32), np.uint32), np.zeros((Ee, Hh, Ii // 128), np.uint16)
     else:
         w13q, w13s = np.zeros((Ee, 2 * Ii, Hh // 8), np.uint32), np.zeros((Ee, 2 * Ii, Hh // 128), np.uint16)
         w2q, w2s = np.zeros((Ee, Hh, Ii // 8), np.uint32), np.zeros((Ee, Hh, Ii // 128), np.uint16)
@@ -591,12 +696,24 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
         if nvfp4:
             a, b = quantize_nvfp4(r13), quantize_nvfp4(r2)
             w13q[e], w13s[e], w13g[e], w2q[e], w2s[e], w2g[e] = a[0][0], a[1][0], a[2][0], b[0][0], b[1][0], b[2][0]
+        elif bitplane:
+            a, b = pack_bitplanes(r13), pack_bitplanes(r2)
+            w13q[e], w13s[e], w2q[e], w2s[e] = a[0][0], a[1][0], b[0][0], b[1][0]
         else:
             a, b = quantize_w4g128(r13), quantize_w4g128(r2)
             w13q[e], w13s[e], w2q[e], w2s[e] = a[0][0], a[1][0], b[0][0], b[1][0]
-    ex = Experts(FMT_NVFP4, w13q, w13s, w2q, w2s, w13g, w2g) if nvfp4 else Experts(FMT_W4G128, w13q, w13s, w2q, w2s)
+    if nvfp4:
+        ex = Experts(FMT_NVFP4, w13q, w13s, w2q, w2s, w13g, w2g)
+    else:
+        ex = Experts(FMT_BITPLANE8 if bitplane else FMT_W4G128, w13q, w13s, w2q, w2s)
     t0 = time.perf_counter()
-    moe_layer(x, wr, bias, ex, k, residual_bits=x)
+    if bitplane:
+        # the same per-step path at per-expert widths (every expert at 3 planes, the budget's mean)
+        r = route(x, wr, bias, k, Ee)
+        y = grouped_ffn(x, r.offsets, r.sorted_pair, k, ex, expand_bits(r.ids, np.full(Ee, 3, np.uint8)))
+        combine(y, r.weights, r.pair_to_row, x)
+    else:
+        moe_layer(x, wr, bias, ex, k, residual_bits=x)
     secs = time.perf_counter() - t0
     try:
         from threadpoolctl import threadpool_info
@@ -649,6 +766,8 @@ def prefill_sample_tokens(cfg) -> int:
     # bounded: a few to about 30 s of oracle work (the NVFP4 oracle decodes element by element)
     if cfg.get("fmt") == "nvfp4":
         return 1
+    if cfg.get("fmt") == "bitplane":
+        return 16
     return 2 if cfg["H"] > 4096 else 32
 
 
@@ -657,7 +776,8 @@ def cpu_baseline_prefill(cfg, seed: int):
     v, secs, thr = oracle_prefill_sample(cfg, n, seed)
     return {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
             "sample": f"{n} tokens through the layer ({secs:.1f} s of CPU work: routing, dequantisation of "
-                      f"their experts, SwiGLU, combine); weights generated and quantised untimed"}
+                      f"their experts" + (" at 3 planes each" if cfg.get("fmt") == "bitplane" else "")
+                      + ", SwiGLU, combine); weights generated and quantised untimed"}
 
 
 def cpu_baseline(batch: int, seed: int):

@@ -25,10 +25,18 @@ enum { kGateUp = 0, kDown = 1 };
 constexpr int kRows = 16;     // weight rows per unit
 constexpr int kWarps = 4;     // warps per CTA, each owning whole units
 constexpr int kThreads = 32 * kWarps;
-constexpr int kDepth = 6;     // group steps in flight per warp (bitplane, NVFP4)
+constexpr int kDepth = 6;     // group steps in flight per warp (NVFP4)
 constexpr int kDepthW4 = 6;   // W4: groups in flight per warp, consumed and refilled two at a time
 constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
 constexpr size_t kSmemTarget = 55 * 1024;  // four CTAs per SM
+// Bitplanes: a group step holds only the planes the chunk reads (b x 16 rows x 16 bytes),
+// so a fixed per-warp ring of 24 plane slots is 8 steps deep at b <= 3, 6 at b = 4, 4 at
+// b = 5..6 and 3 at b = 7..8; two CTAs per SM leave room to stage 16 tokens at K = 2048.
+constexpr int kRingBP = 24 * kRows * 16;
+constexpr size_t kSmemTargetBP = 110 * 1024;
+__host__ __device__ constexpr int bp_depth(int nplanes) {
+  return nplanes <= 3 ? 8 : (nplanes == 4 ? 6 : (nplanes <= 6 ? 4 : 3));
+}
 
 struct FfnArgs {
   const void* act;  // gate/up: x bf16 [T][K]; down: h [P][K] (bf16, or fp16*2^-8 for NVFP4)
@@ -54,8 +62,12 @@ __host__ __device__ constexpr int depth_of() {
   return FMT == MOE_FMT_W4G128 ? kDepthW4 : kDepth;
 }
 template <int FMT>
-__host__ __device__ inline int slot_bytes_of() {  // one group step of one unit
+__host__ __device__ inline int slot_bytes_of() {  // one group step of one unit (bitplanes: all 8 planes)
   return FMT == MOE_FMT_BITPLANE8 ? 8 * kRows * 16 : (FMT == MOE_FMT_NVFP4 ? kRows * 64 + kRows * 8 : kRows * 64);
+}
+template <int FMT>
+__host__ __device__ inline int ring_bytes_of() {  // one warp's ring of group slots
+  return FMT == MOE_FMT_BITPLANE8 ? kRingBP : depth_of<FMT>() * slot_bytes_of<FMT>();
 }
 // x rows: stride/16 = 4 (mod 8) keeps the 8 lanes of a quarter warp on distinct banks
 __host__ __device__ inline int stride_16B(int row_bytes) {
@@ -70,7 +82,6 @@ MOE_DEVICE void cp_async8(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
 MOE_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-MOE_DEVICE void cp_async_wait_depth() { asm volatile("cp.async.wait_group %0;" ::"n"(kDepth - 1) : "memory"); }
 template <int N>
 MOE_DEVICE void cp_async_wait_n() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -128,66 +139,112 @@ MOE_DEVICE void w4h_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa,
   }
 }
 
-// Bitplanes: plane-word bit j <-> element j of the slice.  Bits j and j+16 move to
-// bit 7 / 23 of a bf16x2 whose other bits spell 0.5, so A = 0.5 + 0.5 * bit; the
-// activations were paired (j, j+16) when staged.  With T_p the plane-p MMA sum and X
-// the group sum of the activations, a token read at b planes gets
-//   sum_{p < b} 2^(8-p) T_p + (c_b + 2^(8-b) - 384) X  =  sum_k (u'_k - 128) x_k,
-// c_b = 2^(7-b) for b < 8, 0 for b = 8 (floor plus half-step compensation).
-MOE_DEVICE uint32_t bit_pair(uint32_t w, int j) {
-  const uint32_t s = (j <= 7) ? (w << (7 - j)) : (w >> (j - 7));
-  return (s & 0x00800080u) | 0x3F003F00u;
+// Bitplanes: plane-word bit j <-> element j of the lane's 32-element slice; MMA step s
+// pairs bits (j, j+16) for j = 2s, 2s+1 into one bf16x2 A register (the activations were
+// staged in the same pairing).  Plane p's register is bf16(2^(7-p)) in both halves with
+// the plane bit OR-ed into a mantissa or the sign bit, so A = 2^(7-p) (1 + g_j bit):
+//   j = 0..6   the bit stays in place (mantissa bit j):       g_j = 2^(j-7)
+//   j = 7..14  the bit moves to mantissa bit 6 (one shift):    g_j = 1/2
+//   j = 15     the bit stays in place (the sign):              g_j = -2
+// With the activations staged as x'_k = x_k / g_j(k) (exact: powers of two), one
+// accumulator collects every plane:  T = sum_{p<b} 2^(7-p) (X' + sum_k bit_pk x_k),
+// X' = sum_k x'_k, so that, with X = sum_k x_k and u' the b-bit floor-and-compensation
+// code (floor = sum_{p<b} 2^(7-p) bit_p, compensation c_b = 2^(7-b) for b < 8, 0 for 8),
+//   sum_k (u'_k - 128) x_k = T - (256 - 2^(8-b)) X' + (c_b - 128) X.
+template <int J>
+MOE_DEVICE uint32_t bp_a(uint32_t w, uint32_t base) {
+  if constexpr (J <= 6) return (w & (0x00010001u << J)) | base;
+  else if constexpr (J == 15) return (w & 0x80008000u) | base;
+  else return ((w >> (J - 6)) & 0x00400040u) | base;
 }
-MOE_DEVICE float plane_coef_x(int b) { return (b >= 8) ? -383.f : float(3 * (1 << (7 - b)) - 384); }
+// activation scale 1 / g_j of pair j
+MOE_DEVICE float bp_xscale(int j) { return j <= 6 ? float(1 << (7 - j)) : (j == 15 ? -0.5f : 2.f); }
 
-// pl: the thread's word of plane 0, row g; planes are 16 rows x 16 bytes apart.
+// Widths of the chunk's tokens as one lane sees them: the C columns 2c, 2c+1 (+8) for
+// the epilogue, the B column g (+8) for the tail planes, and the chunk's min / max.
+struct BpChunk {
+  int nplanes, pmin;
+  int bt[2][2];
+  int bB[2];
+};
+
+// one plane of one group: 8 MMA steps per n8 tile; MASK zeroes the B columns of tokens
+// narrower than this plane
+template <bool TWO, bool MASK>
+MOE_DEVICE void bp_plane(uint32_t wa, uint32_t wb, int p, const uint4 (&xv)[2][4], const BpChunk& bc,
+                         float (&t0)[2][4], float (&t1)[2][4]) {
+  const uint32_t e = uint32_t(134 - p) << 7;  // bf16 2^(7-p)
+  const uint32_t base = e | (e << 16);
+  bool keep[2] = {true, true};
+  if (MASK) {
+    keep[0] = p < bc.bB[0];
+    keep[1] = p < bc.bB[1];
+  }
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    uint32_t a0, a1, a2, a3;
+#define MOE_BP_STEP(S)                                         \
+  case S:                                                      \
+    a0 = bp_a<2 * S>(wa, base), a2 = bp_a<2 * S + 1>(wa, base); \
+    a1 = bp_a<2 * S>(wb, base), a3 = bp_a<2 * S + 1>(wb, base); \
+    break;
+    switch (s) {
+      MOE_BP_STEP(0)
+      MOE_BP_STEP(1)
+      MOE_BP_STEP(2)
+      MOE_BP_STEP(3)
+      MOE_BP_STEP(4)
+      MOE_BP_STEP(5)
+      MOE_BP_STEP(6)
+      default:
+        a0 = bp_a<14>(wa, base), a2 = bp_a<15>(wa, base);
+        a1 = bp_a<14>(wb, base), a3 = bp_a<15>(wb, base);
+        break;
+    }
+#undef MOE_BP_STEP
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      if (nt == 1 && !TWO) break;
+      const uint4 xx = xv[nt][s >> 1];
+      uint32_t b0 = (s & 1) ? xx.z : xx.x, b1 = (s & 1) ? xx.w : xx.y;
+      if (MASK && !keep[nt]) b0 = b1 = 0u;
+      float(&t)[4] = (s & 1) ? t1[nt] : t0[nt];
+      mma_bf16(t, a0, a1, a2, a3, b0, b1);
+    }
+  }
+}
+
+// pl: the lane's word of plane 0, row g; planes are 16 rows x 16 bytes apart.  X / X2:
+// the group sums X and X' of the lane's C columns.
 template <bool TWO>
-MOE_DEVICE void bp_group(const uint8_t* pl, int nplanes, const uint4 (&xv)[2][4], const int (&bt)[2][2], float sa,
-                         float sb, const float (&X)[2][2], float (&acc)[2][4]) {
-  constexpr bool two = TWO;
-  float grp[2][4];
+MOE_DEVICE void bp_group(const uint8_t* pl, const BpChunk& bc, const uint4 (&xv)[2][4], float sa, float sb,
+                         const float (&X)[2][2], const float (&X2)[2][2], float (&acc)[2][4]) {
+  float t0[2][4], t1[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) grp[nt][i] = 0.f;
-  for (int p = 0; p < nplanes; ++p) {
-    const uint32_t wa = *reinterpret_cast<const uint32_t*>(pl + p * kRows * 16);
-    const uint32_t wb = *reinterpret_cast<const uint32_t*>(pl + p * kRows * 16 + 8 * 16);
-    float t0[2][4], t1[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) t0[nt][i] = t1[nt][i] = 0.f;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t a0 = bit_pair(wa, 2 * s), a2 = bit_pair(wa, 2 * s + 1);
-      const uint32_t a1 = bit_pair(wb, 2 * s), a3 = bit_pair(wb, 2 * s + 1);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        if (nt == 1 && !two) break;
-        const uint4 xx = xv[nt][s >> 1];
-        const uint32_t b0 = (s & 1) ? xx.z : xx.x, b1 = (s & 1) ? xx.w : xx.y;
-        float(&t)[4] = (s & 1) ? t1[nt] : t0[nt];
-        mma_bf16(t, a0, a1, a2, a3, b0, b1);
-      }
-    }
-    const float f = float(1 << (8 - p));
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const float f0 = (p < bt[nt][0]) ? f : 0.f, f1 = (p < bt[nt][1]) ? f : 0.f;
-      grp[nt][0] = fmaf(f0, t0[nt][0] + t1[nt][0], grp[nt][0]);
-      grp[nt][1] = fmaf(f1, t0[nt][1] + t1[nt][1], grp[nt][1]);
-      grp[nt][2] = fmaf(f0, t0[nt][2] + t1[nt][2], grp[nt][2]);
-      grp[nt][3] = fmaf(f1, t0[nt][3] + t1[nt][3], grp[nt][3]);
-    }
-  }
+    for (int i = 0; i < 4; ++i) t0[nt][i] = t1[nt][i] = 0.f;
+  int p = 0;
+  for (; p < bc.pmin; ++p)  // planes every token of the chunk reads
+    bp_plane<TWO, false>(*reinterpret_cast<const uint32_t*>(pl + p * kRows * 16),
+                         *reinterpret_cast<const uint32_t*>(pl + p * kRows * 16 + 8 * 16), p, xv, bc, t0, t1);
+  for (; p < bc.nplanes; ++p)  // planes only the wider tokens read
+    bp_plane<TWO, true>(*reinterpret_cast<const uint32_t*>(pl + p * kRows * 16),
+                        *reinterpret_cast<const uint32_t*>(pl + p * kRows * 16 + 8 * 16), p, xv, bc, t0, t1);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    const float x0 = plane_coef_x(bt[nt][0]) * X[nt][0], x1 = plane_coef_x(bt[nt][1]) * X[nt][1];
-    acc[nt][0] = fmaf(sa, grp[nt][0] + x0, acc[nt][0]);
-    acc[nt][1] = fmaf(sa, grp[nt][1] + x1, acc[nt][1]);
-    acc[nt][2] = fmaf(sb, grp[nt][2] + x0, acc[nt][2]);
-    acc[nt][3] = fmaf(sb, grp[nt][3] + x1, acc[nt][3]);
+    if (nt == 1 && !TWO) break;
+    float corr[2];
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int b = bc.bt[nt][jj];
+      const float k1 = float(256 - (1 << (8 - b))), k2 = float((b < 8 ? (1 << (7 - b)) : 0) - 128);
+      corr[jj] = fmaf(k2, X[nt][jj], -k1 * X2[nt][jj]);
+    }
+    acc[nt][0] = fmaf(sa, (t0[nt][0] + t1[nt][0]) + corr[0], acc[nt][0]);
+    acc[nt][1] = fmaf(sa, (t0[nt][1] + t1[nt][1]) + corr[1], acc[nt][1]);
+    acc[nt][2] = fmaf(sb, (t0[nt][2] + t1[nt][2]) + corr[0], acc[nt][2]);
+    acc[nt][3] = fmaf(sb, (t0[nt][3] + t1[nt][3]) + corr[1], acc[nt][3]);
   }
 }
 
@@ -268,20 +325,20 @@ MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* 
 }
 
 // ---------------------------------------------------------------- one unit (bitplane, NVFP4)
-// Streams the warp's unit: for G = 0 .. GK-1, waits for group G's slot, computes it
-// against the staged activations of one (TWO = false) or two n8 token tiles, and refills
-// the slot with group G + kDepth.
-template <int FMT, bool TWO, class Issue>
-MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t* wscale, const uint8_t* xbuf,
-                            const float* xsum, int GK, int g, int c, int nvalid, int nplanes, const int (&bt)[2][2],
-                            Issue&& issue, float (&acc)[2][4]) {
+// Streams the warp's unit through a ring of D slots of `slot` bytes: for G = 0 .. GK-1,
+// waits for group G's slot, computes it against the staged activations of one (TWO =
+// false) or two n8 token tiles, and refills the slot with group G + D.
+template <int FMT, bool TWO, int D, class Issue>
+MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, int slot, const uint16_t* wscale,
+                            const uint8_t* xbuf, const float* xsum, int GK, int g, int c, int nvalid,
+                            const BpChunk& bc, Issue&& issue, float (&acc)[2][4]) {
   constexpr int NT = TWO ? 2 : 1;
   for (int G = 0; G < GK; ++G) {
-    cp_async_wait_depth();
+    cp_async_wait_n<D - 1>();
     __syncwarp();  // every lane's copies of group G have landed
-    const uint8_t* sl = wsm + (G % kDepth) * a.slot_bytes;
+    const uint8_t* sl = wsm + (G % D) * slot;
     uint4 xv[2][4];
-    float X[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    float X[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, X2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       // B column of an absent token: any staged row will do (each output column depends
@@ -290,15 +347,18 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t
       const uint8_t* xr = xbuf + size_t(row) * a.x_stride + G * 256 + c * 16;
 #pragma unroll
       for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
-      if (FMT != MOE_FMT_NVFP4) {  // group sums of C columns 2c, 2c+1 ([G][kMaxTok] staged)
-        const float2 x2 = *reinterpret_cast<const float2*>(xsum + G * kMaxTok + nt * 8 + 2 * c);
-        X[nt][0] = x2.x;
-        X[nt][1] = x2.y;
+      if (FMT == MOE_FMT_BITPLANE8) {  // group sums X, X' of C columns 2c, 2c+1 ([G][kMaxTok] each)
+        const float2 x1 = *reinterpret_cast<const float2*>(xsum + G * kMaxTok + nt * 8 + 2 * c);
+        const float2 x2 = *reinterpret_cast<const float2*>(xsum + (GK + G) * kMaxTok + nt * 8 + 2 * c);
+        X[nt][0] = x1.x;
+        X[nt][1] = x1.y;
+        X2[nt][0] = x2.x;
+        X2[nt][1] = x2.y;
       }
     }
     if (FMT == MOE_FMT_BITPLANE8) {
-      bp_group<TWO>(sl + g * 16 + c * 4, nplanes, xv, bt, bf16_bits_to_float(wscale[g * GK + G]),
-                    bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, acc);
+      bp_group<TWO>(sl + g * 16 + c * 4, bc, xv, bf16_bits_to_float(wscale[g * GK + G]),
+                    bf16_bits_to_float(wscale[(g + 8) * GK + G]), X, X2, acc);
     } else {
       const uint8_t* wr = sl + g * 64 + c * 16;
       const uint8_t* sc = sl + kRows * 64;  // [16 rows][8 block scales]
@@ -308,8 +368,30 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, const uint16_t
                      xv, acc);
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
-    if (G + kDepth < GK) issue(G + kDepth);
+    if (G + D < GK) issue(G + D);
     cp_async_commit();
+  }
+}
+
+// bitplanes: the ring depth for the chunk's prefix length, as a compile-time constant
+template <bool TWO, class Issue>
+MOE_DEVICE void stream_unit_bp(const FfnArgs& a, const uint8_t* wsm, const uint16_t* wscale, const uint8_t* xbuf,
+                               const float* xsum, int GK, int g, int c, int nvalid, const BpChunk& bc,
+                               Issue&& issue, float (&acc)[2][4]) {
+  const int slot = bc.nplanes * kRows * 16;
+  switch (bp_depth(bc.nplanes)) {
+    case 8:
+      stream_unit<MOE_FMT_BITPLANE8, TWO, 8>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+      break;
+    case 6:
+      stream_unit<MOE_FMT_BITPLANE8, TWO, 6>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+      break;
+    case 4:
+      stream_unit<MOE_FMT_BITPLANE8, TWO, 4>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+      break;
+    default:
+      stream_unit<MOE_FMT_BITPLANE8, TWO, 3>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+      break;
   }
 }
 
@@ -333,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
   float* xsum = reinterpret_cast<float*>(smem + a.off_xsum);
   int* sbits = reinterpret_cast<int*>(smem + a.off_bits);
   uint8_t* wsm = smem + size_t(warp) * a.warp_bytes;  // this warp's ring (+ scales)
-  uint16_t* wscale = reinterpret_cast<uint16_t*>(wsm + depth_of<FMT>() * a.slot_bytes);
+  uint16_t* wscale = reinterpret_cast<uint16_t*>(wsm + ring_bytes_of<FMT>());
 
   auto wrow = [&](int i) -> int {  // expert-matrix row of unit row i
     if (MODE == kGateUp) return (i < 8) ? (8 * rt + i) : (a.I + 8 * rt + i - 8);
@@ -368,14 +450,19 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
     const bool two = nvalid > 8;
     if (tok0 > 0) __syncthreads();  // the previous chunk's activations are no longer read
 
-    // bitplanes: prefix length of this chunk (known before any weight is requested)
-    int nplanes = 1;
+    // bitplanes: prefix length of this chunk (known before any weight is requested): lane n
+    // reads token n's width (nvalid <= 16), one warp max-reduction
+    int nplanes = 1, pmin = 1;
     if (FMT == MOE_FMT_BITPLANE8) {
-      for (int n = 0; n < nvalid; ++n) nplanes = max(nplanes, int(a.bits[a.sorted_pair[row0 + tok0 + n]]));
-      nplanes = min(8, nplanes);
+      const int v = (lane < nvalid) ? min(8, max(1, int(a.bits[a.sorted_pair[row0 + tok0 + lane]]))) : 0;
+      nplanes = max(1, __reduce_max_sync(0xffffffffu, v));
+      pmin = __reduce_min_sync(0xffffffffu, lane < nvalid ? v : 8);
     }
-    auto issue = [&](int G) {  // copy group G of the unit into ring slot G % kDepth
-      uint8_t* dst = wsm + (G % depth_of<FMT>()) * a.slot_bytes;
+    // ring geometry of this chunk: bitplane slots hold the chunk's nplanes planes only
+    const int ring_slot = (FMT == MOE_FMT_BITPLANE8) ? nplanes * kRows * 16 : a.slot_bytes;
+    const int ring_depth = (FMT == MOE_FMT_BITPLANE8) ? bp_depth(nplanes) : depth_of<FMT>();
+    auto issue = [&](int G) {  // copy group G of the unit into ring slot G % ring_depth
+      uint8_t* dst = wsm + (G % ring_depth) * ring_slot;
       if (FMT == MOE_FMT_BITPLANE8) {
         const int i = lane & 15;
         for (int p = lane >> 4; p < nplanes; p += 2)
@@ -425,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
           cp_async_commit();
         }
       } else {
-        for (int G = 0; G < kDepth; ++G) {
+        for (int G = 0; G < ring_depth; ++G) {
           if (G < GK) issue(G);
           cp_async_commit();
         }
@@ -438,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
     for (int q0 = 0; q0 < nslices; q0 += kThreads) {
       const int q = q0 + threadIdx.x;
       const bool ok = q < nslices;
-      float ssum = 0.f;
+      float ssum = 0.f, ssum2 = 0.f;
       int n = 0, sl = 0;
       if (ok) {
         n = q / slices;
@@ -479,10 +566,15 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
           }
           ssum = -1032.f * lo - 1152.f * hi;
         } else if (FMT == MOE_FMT_BITPLANE8) {
+          // step s: (x_2s, x_2s+16), (x_2s+1, x_2s+17), each pair j scaled by 1 / g_j (exact)
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {  // step s: (x_2s, x_2s+16), (x_2s+1, x_2s+17)
-            O[2 * s] = __byte_perm(R[s], R[s + 8], 0x5410);
-            O[2 * s + 1] = __byte_perm(R[s], R[s + 8], 0x7632);
+          for (int s = 0; s < 8; ++s) {
+            const float f0 = bp_xscale(2 * s), f1 = bp_xscale(2 * s + 1);
+            const float lo0 = bf16_lo(R[s]) * f0, hi0 = bf16_lo(R[s + 8]) * f0;
+            const float lo1 = bf16_hi(R[s]) * f1, hi1 = bf16_hi(R[s + 8]) * f1;
+            O[2 * s] = uint32_t(float_to_bf16_bits(lo0)) | (uint32_t(float_to_bf16_bits(hi0)) << 16);
+            O[2 * s + 1] = uint32_t(float_to_bf16_bits(lo1)) | (uint32_t(float_to_bf16_bits(hi1)) << 16);
+            ssum2 += (lo0 + hi0) + (lo1 + hi1);
           }
         } else {
           if (MODE == kGateUp) {  // bf16 -> fp16 * 2^-8, natural pairs
@@ -513,19 +605,25 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
         ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
         if (ok && (sl & 3) == 0) xsum[(sl >> 2) * kMaxTok + n] = ssum;
       }
+      if (FMT == MOE_FMT_BITPLANE8) {  // and X' ([GK + G][kMaxTok])
+        ssum2 += __shfl_xor_sync(0xffffffffu, ssum2, 1);
+        ssum2 += __shfl_xor_sync(0xffffffffu, ssum2, 2);
+        if (ok && (sl & 3) == 0) xsum[(slices / 4 + (sl >> 2)) * kMaxTok + n] = ssum2;
+      }
     }
     if (FMT == MOE_FMT_BITPLANE8)
       for (int n = threadIdx.x; n < kMaxTok; n += kThreads)
-        sbits[n] = (n < nvalid) ? int(a.bits[a.sorted_pair[row0 + tok0 + n]]) : 8;
+        sbits[n] = (n < nvalid) ? min(8, max(1, int(a.bits[a.sorted_pair[row0 + tok0 + n]]))) : 8;
     __syncthreads();
     if (!has_unit) continue;
 
-    int bt[2][2] = {{8, 8}, {8, 8}};
+    BpChunk bc{nplanes, pmin, {{8, 8}, {8, 8}}, {8, 8}};
     if (FMT == MOE_FMT_BITPLANE8) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        bt[nt][0] = sbits[nt * 8 + 2 * c];
-        bt[nt][1] = sbits[nt * 8 + 2 * c + 1];
+        bc.bt[nt][0] = sbits[nt * 8 + 2 * c];
+        bc.bt[nt][1] = sbits[nt * 8 + 2 * c + 1];
+        bc.bB[nt] = sbits[nt * 8 + g];
       }
     }
 
@@ -535,15 +633,23 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    if (FMT == MOE_FMT_W4G128) {
+    if constexpr (FMT == MOE_FMT_W4G128) {
       if (two)
         stream_w4<true>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, issue, acc);
       else
         stream_w4<false>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, issue, acc);
-    } else if (two) {
-      stream_unit<FMT, true>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, nplanes, bt, issue, acc);
+    } else if constexpr (FMT == MOE_FMT_BITPLANE8) {
+      if (two)
+        stream_unit_bp<true>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+      else
+        stream_unit_bp<false>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
     } else {
-      stream_unit<FMT, false>(a, wsm, wscale, xbuf, xsum, GK, g, c, nvalid, nplanes, bt, issue, acc);
+      if (two)
+        stream_unit<FMT, true, kDepth>(a, wsm, a.slot_bytes, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue,
+                                       acc);
+      else
+        stream_unit<FMT, false, kDepth>(a, wsm, a.slot_bytes, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue,
+                                        acc);
     }
     cp_async_wait_all();
 
@@ -589,10 +695,12 @@ static bool plan(FfnArgs& a) {
   const int K = a.K, GK = K / 128;
   a.slot_bytes = slot_bytes_of<FMT>();
   const int scale_bytes = (FMT == MOE_FMT_NVFP4) ? 0 : int(align256(size_t(kRows) * GK * 2));
-  a.warp_bytes = int(align256(size_t(depth_of<FMT>()) * a.slot_bytes + scale_bytes));
+  a.warp_bytes = int(align256(size_t(ring_bytes_of<FMT>()) + scale_bytes));
   a.x_stride = stride_16B(K * 2);
-  const size_t fixed = size_t(kWarps) * a.warp_bytes + align256(size_t(kMaxTok) * GK * 4) + 256;
-  const size_t room = fixed < kSmemTarget ? kSmemTarget - fixed : 0;
+  const int nsum = (FMT == MOE_FMT_BITPLANE8) ? 2 : 1;  // bitplanes: X and X'
+  const size_t fixed = size_t(kWarps) * a.warp_bytes + align256(size_t(nsum) * kMaxTok * GK * 4) + 256;
+  const size_t target = (FMT == MOE_FMT_BITPLANE8) ? kSmemTargetBP : kSmemTarget;
+  const size_t room = fixed < target ? target - fixed : 0;
   int nx = int(room / size_t(a.x_stride));
   nx = nx < 1 ? 1 : nx;  // wide rows: at least one token row (then one CTA per SM)
   a.nx = nx > kMaxTok ? kMaxTok : nx;
@@ -600,7 +708,7 @@ static bool plan(FfnArgs& a) {
   a.off_x = int(off);
   off += align256(size_t(a.nx) * a.x_stride);
   a.off_xsum = int(off);
-  off += align256(size_t(kMaxTok) * GK * 4);
+  off += align256(size_t(nsum) * kMaxTok * GK * 4);
   a.off_bits = int(off);
   off += 256;
   return off <= 220 * 1024;
