@@ -23,19 +23,23 @@ namespace moe {
 
 enum { kGateUp = 0, kDown = 1 };
 constexpr int kRows = 16;     // weight rows per unit
-constexpr int kWarps = 4;     // warps per CTA, each owning whole units
+constexpr int kWarps = 4;     // warps per CTA (W4, NVFP4), each owning whole units
 constexpr int kThreads = 32 * kWarps;
+constexpr int kWarpsBP = 8;   // bitplanes: eight warps share one activation stage
 constexpr int kDepth = 6;     // group steps in flight per warp (NVFP4)
 constexpr int kDepthW4 = 6;   // W4: groups in flight per warp, consumed and refilled two at a time
 constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
 constexpr size_t kSmemTarget = 55 * 1024;  // four CTAs per SM
 // Bitplanes: a group step holds only the planes the chunk reads (b x 16 rows x 16 bytes),
-// so a fixed per-warp ring of 24 plane slots is 8 steps deep at b <= 3, 6 at b = 4, 4 at
-// b = 5..6 and 3 at b = 7..8; two CTAs per SM leave room to stage 16 tokens at K = 2048.
-constexpr int kRingBP = 24 * kRows * 16;
-constexpr size_t kSmemTargetBP = 110 * 1024;
-__host__ __device__ constexpr int bp_depth(int nplanes) {
-  return nplanes <= 3 ? 8 : (nplanes == 4 ? 6 : (nplanes <= 6 ? 4 : 3));
+// so a fixed per-warp ring of 16 plane slots is min(8, 16 / b) steps deep (8 at b <= 2, 5
+// at b = 3, 4, 3, then 2 at b >= 6); two 8-warp CTAs per SM still stage 16 tokens at
+// K = 2048 (16 warps per SM).
+constexpr int kRingBP = 16 * kRows * 16;
+constexpr size_t kSmemTargetBP = 112 * 1024;
+__host__ __device__ constexpr int bp_depth(int nplanes) { return (16 / nplanes) < 8 ? 16 / nplanes : 8; }
+template <int FMT>
+__host__ __device__ constexpr int warps_of() {
+  return FMT == MOE_FMT_BITPLANE8 ? kWarpsBP : kWarps;
 }
 
 struct FfnArgs {
@@ -383,21 +387,25 @@ MOE_DEVICE void stream_unit_bp(const FfnArgs& a, const uint8_t* wsm, const uint1
     case 8:
       stream_unit<MOE_FMT_BITPLANE8, TWO, 8>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
       break;
-    case 6:
-      stream_unit<MOE_FMT_BITPLANE8, TWO, 6>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+    case 5:
+      stream_unit<MOE_FMT_BITPLANE8, TWO, 5>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
       break;
     case 4:
       stream_unit<MOE_FMT_BITPLANE8, TWO, 4>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
       break;
-    default:
+    case 3:
       stream_unit<MOE_FMT_BITPLANE8, TWO, 3>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
+      break;
+    default:
+      stream_unit<MOE_FMT_BITPLANE8, TWO, 2>(a, wsm, slot, wscale, xbuf, xsum, GK, g, c, nvalid, bc, issue, acc);
       break;
   }
 }
 
 // ---------------------------------------------------------------- kernel
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
+__global__ void __launch_bounds__(32 * warps_of<FMT>(), 16 / warps_of<FMT>()) k_ffn_gemv(FfnArgs a) {
+  constexpr int WARPS = warps_of<FMT>(), THREADS = 32 * WARPS;
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int slot = blockIdx.y;
@@ -408,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   const int K = a.K, GK = K / 128;
   const int TPE = (MODE == kGateUp) ? a.I / 8 : a.N / kRows;
-  const int rt = blockIdx.x * kWarps + warp;  // this warp's unit
+  const int rt = blockIdx.x * WARPS + warp;  // this warp's unit
   const bool has_unit = rt < TPE;
 
   uint8_t* xbuf = smem + a.off_x;
@@ -522,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
     // ---- stage activations: slice q = (token n, 32-element slice sl), pre-paired per format
     const int slices = K / 32;
     const int nslices = nvalid * slices;
-    for (int q0 = 0; q0 < nslices; q0 += kThreads) {
+    for (int q0 = 0; q0 < nslices; q0 += THREADS) {
       const int q = q0 + threadIdx.x;
       const bool ok = q < nslices;
       float ssum = 0.f, ssum2 = 0.f;
@@ -612,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a) {
       }
     }
     if (FMT == MOE_FMT_BITPLANE8)
-      for (int n = threadIdx.x; n < kMaxTok; n += kThreads)
+      for (int n = threadIdx.x; n < kMaxTok; n += THREADS)
         sbits[n] = (n < nvalid) ? min(8, max(1, int(a.bits[a.sorted_pair[row0 + tok0 + n]]))) : 8;
     __syncthreads();
     if (!has_unit) continue;
@@ -698,13 +706,13 @@ static bool plan(FfnArgs& a) {
   a.warp_bytes = int(align256(size_t(ring_bytes_of<FMT>()) + scale_bytes));
   a.x_stride = stride_16B(K * 2);
   const int nsum = (FMT == MOE_FMT_BITPLANE8) ? 2 : 1;  // bitplanes: X and X'
-  const size_t fixed = size_t(kWarps) * a.warp_bytes + align256(size_t(nsum) * kMaxTok * GK * 4) + 256;
+  const size_t fixed = size_t(warps_of<FMT>()) * a.warp_bytes + align256(size_t(nsum) * kMaxTok * GK * 4) + 256;
   const size_t target = (FMT == MOE_FMT_BITPLANE8) ? kSmemTargetBP : kSmemTarget;
   const size_t room = fixed < target ? target - fixed : 0;
   int nx = int(room / size_t(a.x_stride));
   nx = nx < 1 ? 1 : nx;  // wide rows: at least one token row (then one CTA per SM)
   a.nx = nx > kMaxTok ? kMaxTok : nx;
-  size_t off = size_t(kWarps) * a.warp_bytes;
+  size_t off = size_t(warps_of<FMT>()) * a.warp_bytes;
   a.off_x = int(off);
   off += align256(size_t(a.nx) * a.x_stride);
   a.off_xsum = int(off);
@@ -731,7 +739,8 @@ static cudaError_t launch_one(FfnArgs a, int slots, cudaStream_t st) {
     raised[dev] = true;
   }
   const int TPE = (MODE == kGateUp) ? a.I / 8 : a.N / kRows;
-  k_ffn_gemv<FMT, MODE><<<dim3(unsigned((TPE + kWarps - 1) / kWarps), unsigned(slots)), kThreads, smem, st>>>(a);
+  constexpr int W = warps_of<FMT>();
+  k_ffn_gemv<FMT, MODE><<<dim3(unsigned((TPE + W - 1) / W), unsigned(slots)), 32 * W, smem, st>>>(a);
   return cudaGetLastError();
 }
 
