@@ -64,6 +64,10 @@ _SIGS = {
     "moe_allocate_bits": ([_vp, _vp, _vp, _i64, _i64, ctypes.POINTER(ctypes.c_uint8), _i64, _d, _vp, _vp, _vp],
                           ctypes.c_int),
     "moe_expand_bits": ([_vp, _vp, _i64, _i64, _vp, _vp], ctypes.c_int),
+    "moe_cache_state_bytes": ([_i64, _i64], _sz),
+    "moe_cache_init": ([_vp, _sz, _i64, _i64, _i64], ctypes.c_int),
+    "moe_cache_plan": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+    "moe_cache_slots": ([_vp, _vp, _vp], ctypes.c_int),
     "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
     "moe_grouped_ffn": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
                          _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
@@ -267,6 +271,53 @@ def moe_expand_bits(topk_ids: torch.Tensor, bits_e: torch.Tensor, k: int, bits: 
     bits = torch.empty(max(n, 1), dtype=torch.uint8, device=topk_ids.device) if bits is None else bits
     _call("moe_expand_bits", _p(topk_ids), _p(bits_e), n // k, k, _p(bits), _stream(stream))
     return bits
+
+
+# ---------------------------------------------------------------- expert slot cache (host planning)
+def _hp(a) -> int:
+    """Address of a C-contiguous host numpy array (the cache entry points take host memory)."""
+    import numpy as np
+    if not isinstance(a, np.ndarray) or not a.flags["C_CONTIGUOUS"]:
+        raise ValueError("expected a C-contiguous numpy array")
+    return a.ctypes.data
+
+
+def moe_cache_state_bytes(E: int, S: int) -> int:
+    return int(load().moe_cache_state_bytes(E, S))
+
+
+def moe_cache_init(E: int, S: int, planes: int):
+    """A fresh cache state (host numpy buffer) of S slots over E experts."""
+    import numpy as np
+    nbytes = moe_cache_state_bytes(E, S)
+    if nbytes == 0:
+        raise MoeError("moe_cache_state_bytes", 1)
+    state = np.zeros((nbytes + 7) // 8, dtype=np.int64)
+    _call("moe_cache_init", _hp(state), state.nbytes, E, S, planes)
+    return state
+
+
+def moe_cache_plan(state, need):
+    """Plan one step: returns (served_expert, served_slot, fetch_lo, fetch_hi, round_start)
+    as numpy arrays, round_start of length R + 1."""
+    import numpy as np
+    need = np.ascontiguousarray(need, dtype=np.uint8)
+    E = need.size
+    se, ss = np.zeros(E, np.int32), np.zeros(E, np.int32)
+    lo, hi = np.zeros(E, np.uint8), np.zeros(E, np.uint8)
+    rs = np.zeros(E + 1, np.int32)
+    nr = ctypes.c_int32(0)
+    _call("moe_cache_plan", _hp(state), _hp(need), _hp(se), _hp(ss), _hp(lo), _hp(hi), _hp(rs), ctypes.byref(nr))
+    n = int(rs[nr.value])
+    return se[:n], ss[:n], lo[:n], hi[:n], rs[:nr.value + 1]
+
+
+def moe_cache_slots(state, S: int):
+    """(expert_of int32 [S], planes uint8 [S]) of a cache state."""
+    import numpy as np
+    eo, pl = np.zeros(S, np.int32), np.zeros(S, np.uint8)
+    _call("moe_cache_slots", _hp(state), _hp(eo), _hp(pl))
+    return eo, pl
 
 
 # ---------------------------------------------------------------- FFN and combine

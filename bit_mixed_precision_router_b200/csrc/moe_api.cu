@@ -5,6 +5,7 @@
 
 #include <climits>
 
+#include "moe_cache_core.cuh"
 #include "moe_common.cuh"
 #include "moe_internal.h"
 #include "moe_synth.h"
@@ -171,6 +172,55 @@ moe_status_t moe_expand_bits(const int32_t* topk_ids, const uint8_t* bits_e, int
   if (!topk_ids || !bits_e || !bits) return MOE_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(topk_ids) & 3u) return MOE_ERR_MISALIGNED;
   return from_cuda(moe::launch_expand_bits(topk_ids, bits_e, T * k, bits, as_stream(stream)));
+}
+
+size_t moe_cache_state_bytes(int64_t E, int64_t S) {
+  if (E < 1 || E > MOE_MAX_EXPERTS || S < 1 || S > E) return 0;
+  return moe::cache_state_bytes(int(E), int(S));
+}
+
+moe_status_t moe_cache_init(void* state, size_t state_bytes, int64_t E, int64_t S, int64_t planes) {
+  if (!state) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > MOE_MAX_EXPERTS || S < 1 || S > E || planes < 1 || planes > 8) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(state) & 7u) return MOE_ERR_MISALIGNED;
+  if (state_bytes < moe::cache_state_bytes(int(E), int(S))) return MOE_ERR_WORKSPACE;
+  moe::cache_reset(moe::cache_view(state, int(E), int(S)), int(E), int(S), int(planes));
+  return MOE_OK;
+}
+
+static moe_status_t cache_header(const void* state, const moe::CacheHeader** h) {
+  if (!state) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(state) & 7u) return MOE_ERR_MISALIGNED;
+  *h = static_cast<const moe::CacheHeader*>(state);
+  if ((*h)->magic != moe::kCacheMagic) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status_t moe_cache_plan(void* state, const uint8_t* need, int32_t* served_expert, int32_t* served_slot,
+                            uint8_t* fetch_lo, uint8_t* fetch_hi, int32_t* round_start, int32_t* nrounds) {
+  const moe::CacheHeader* h = nullptr;
+  const moe_status_t st = cache_header(state, &h);
+  if (st != MOE_OK) return st;
+  if (!need || !served_expert || !served_slot || !fetch_lo || !fetch_hi || !round_start || !nrounds)
+    return MOE_ERR_INVALID_ARG;
+  for (int e = 0; e < h->E; ++e)  // validated before the state changes
+    if (need[e] > h->P) return MOE_ERR_INVALID_ARG;
+  *nrounds = moe::cache_plan(moe::cache_view(state, h->E, h->S), need, served_expert, served_slot, fetch_lo,
+                             fetch_hi, round_start);
+  return MOE_OK;
+}
+
+moe_status_t moe_cache_slots(const void* state, int32_t* expert_of, uint8_t* planes) {
+  const moe::CacheHeader* h = nullptr;
+  const moe_status_t st = cache_header(state, &h);
+  if (st != MOE_OK) return st;
+  if (!expert_of || !planes) return MOE_ERR_INVALID_ARG;
+  const moe::CacheView v = moe::cache_view(const_cast<void*>(state), h->E, h->S);
+  for (int s = 0; s < h->S; ++s) {
+    expert_of[s] = v.expert_of[s];
+    planes[s] = v.planes[s];
+  }
+  return MOE_OK;
 }
 
 moe_status_t moe_select_bits(const float* topk_w, int64_t T, int64_t k, const float thresholds[3],

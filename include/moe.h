@@ -237,6 +237,46 @@ moe_status_t moe_allocate_bits(const double* delta, const double* m, const int32
 moe_status_t moe_expand_bits(const int32_t* topk_ids, const uint8_t* bits_e, int64_t T, int64_t k,
                              uint8_t* bits, moe_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Expert slot cache: planning (HOST functions: host memory only, no CUDA call)
+ * [ExactMoE abstract: routed experts kept in pinned host memory and executed through a
+ * configurable GPU-resident slot cache, every routed expert served; PagedMoE abstract:
+ * a cached bitplane prefix is reused or extended by fetching only the missing planes,
+ * the prefix length decided before any transfer].
+ *
+ * A step's demand need[e] (0 = nothing routed to e; else the planes its pairs read,
+ * 1..planes) is served in ascending expert id:
+ *   hit        resident with >= need[e] planes: nothing fetched;
+ *   extension  resident with h < need[e] planes: fetch planes [h, need[e]);
+ *   miss       fetch planes [0, need[e]) into the lowest free slot, else into the slot,
+ *              among those not served in the current round, with the smallest
+ *              (holds an expert needed later in the step, last step used, slot index).
+ * When a miss finds every slot served in the current round, the round closes (the
+ * caller computes its experts) and a new round starts; a step needing <= S experts is
+ * one round.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of host memory for the state of a cache of S slots over E experts; 0 if
+ * 1 <= S <= E <= MOE_MAX_EXPERTS does not hold. */
+size_t moe_cache_state_bytes(int64_t E, int64_t S);
+
+/* Initialise a cache state (all slots free) in caller-owned host memory, 8-byte aligned,
+ * of at least moe_cache_state_bytes(E, S) bytes.  planes: 8 for bitplane experts, 1 for
+ * whole-expert formats (W4 g128, NVFP4).  MOE_ERR_WORKSPACE if state_bytes is short. */
+moe_status_t moe_cache_init(void* state, size_t state_bytes, int64_t E, int64_t S, int64_t planes);
+
+/* Plan one step and update the state (host arrays throughout).  need uint8 [E], each
+ * <= planes (checked before the state changes).  Outputs for the n routed experts, in
+ * service order: served_expert int32 [n], served_slot int32 [n], fetch_lo / fetch_hi
+ * uint8 [n] (planes [lo, hi) to copy into the slot; lo == hi: nothing); round_start
+ * int32 [R + 1] (round r = entries [round_start[r], round_start[r+1])); *nrounds = R.
+ * Capacities: E entries for the per-expert arrays, E + 1 for round_start. */
+moe_status_t moe_cache_plan(void* state, const uint8_t* need, int32_t* served_expert, int32_t* served_slot,
+                            uint8_t* fetch_lo, uint8_t* fetch_hi, int32_t* round_start, int32_t* nrounds);
+
+/* The slots' contents: expert_of int32 [S] (-1 = free) and resident planes uint8 [S]. */
+moe_status_t moe_cache_slots(const void* state, int32_t* expert_of, uint8_t* planes);
+
 /* Per-pair bit-width from the routing weight [MatMoE: precision per expert from
  * routing scores; PagedMoE: prefix length from current routing weights].
  * bits[p] = choices[0] if w < thresholds[0], choices[1] if w < thresholds[1],
