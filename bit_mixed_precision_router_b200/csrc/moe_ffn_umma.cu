@@ -57,7 +57,7 @@ constexpr int kWStages = 4;     // packed-weight stages in shared memory
 constexpr int kAStages = 2;     // dequantised weight stages in tensor memory (64 columns each)
 constexpr int kDeqSets = 2;     // dequantising warp sets, alternating K blocks
 constexpr int kThreadsU = 32 * (4 + 4 * kDeqSets + 4);
-constexpr int kTmemCols = 512;  // accumulators at columns 0 and 192, A stages at 384 + 32 a
+constexpr int kTmemCols = 512;  // accumulators at columns 0 and 192, A stages at 384 + 64 a
 constexpr int kACol0 = 2 * kTN;
 constexpr int kAtomBytes = kTN * 128;   // one swizzle atom of routed rows
 constexpr int kBStageBytes = 2 * kAtomBytes;
