@@ -1,6 +1,7 @@
 // The C ABI (moe.h, moe_synth.h): host-side argument validation, then dispatch to
 // the launchers.  Nothing here allocates device memory or synchronises, except
 // moe_check_device_errors.
+#include <atomic>
 #include <stdint.h>
 
 #include <climits>
@@ -17,15 +18,18 @@ __device__ unsigned g_moe_error_word;
 namespace moe {
 
 unsigned* device_error_word() {
-  static unsigned* cached[128] = {};
+  // per-device lookup cached on first use (host threads may race to store the same value)
+  static std::atomic<unsigned*> cached[128] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-  if (!cached[dev]) {
+  unsigned* w = cached[dev].load(std::memory_order_relaxed);
+  if (!w) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_moe_error_word) != cudaSuccess) return nullptr;
-    cached[dev] = static_cast<unsigned*>(p);
+    w = static_cast<unsigned*>(p);
+    cached[dev].store(w, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return w;
 }
 
 }  // namespace moe

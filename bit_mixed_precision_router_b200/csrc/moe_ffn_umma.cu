@@ -40,6 +40,7 @@
 //
 // Every wait is bounded (mbar_wait): a wait that runs out sets the device error
 // word and the role stops; the CTA still frees its tensor memory.
+#include <atomic>
 #include <cuda.h>  // CUtensorMap and its enums; the encoder is reached through the runtime
 
 #include "moe_common.cuh"
@@ -616,28 +617,28 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
 }
 
 int sm_count() {
-  static int cached[128] = {};
+  static std::atomic<int> cached[128] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
-  if (!cached[dev]) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 template <int FMT, int MODE>
 cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const UmmaArgs& a, cudaStream_t st) {
-  static bool raised[128] = {};
+  static std::atomic<bool> raised[128] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-  if (!raised[dev]) {
+  if (!raised[dev].load(std::memory_order_relaxed)) {
     const cudaError_t err =
         cudaFuncSetAttribute(k_ffn_umma<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    raised[dev] = true;
+    raised[dev].store(true, std::memory_order_relaxed);
   }
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;

@@ -7,6 +7,8 @@
 // One warp evaluates a 4-token x 8-expert tile: lane L holds partial L of all 32
 // logits, and a recursive-halving exchange (which adds exactly the same pairs as
 // the pairwise tree) leaves logit (t, e) = (L / 8, L % 8) in lane L.
+#include <atomic>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -383,13 +385,13 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
     const size_t perm = size_t(((T * k + 3) & ~3) + kFusedWarps * E + E) * 4;
     const size_t smem = stage > perm ? stage : perm;
     if (smem > 48 * 1024) {
-      static bool raised[128] = {};
+      static std::atomic<bool> raised[128] = {};
       int dev = 0;
       cudaGetDevice(&dev);
-      if (dev >= 0 && dev < 128 && !raised[dev]) {
+      if (dev >= 0 && dev < 128 && !raised[dev].load(std::memory_order_relaxed)) {
         err = cudaFuncSetAttribute(k_route_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
         if (err != cudaSuccess) return err;
-        raised[dev] = true;
+        raised[dev].store(true, std::memory_order_relaxed);
       }
     }
     k_route_fused<<<dim3(unsigned((E + kFusedWarps - 1) / kFusedWarps)), 32 * kFusedWarps, smem, st>>>(

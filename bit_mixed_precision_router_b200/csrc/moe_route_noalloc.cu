@@ -24,6 +24,7 @@
 // cudaGetSymbolAddress (the host-side name is only a stand-in, never a device
 // address) while that device is current, and caches it per device.  Make that
 // first call before capturing a stream into a graph.
+#include <atomic>
 #include <climits>
 
 #include "moe_common.cuh"
@@ -37,15 +38,17 @@ static __device__ __align__(256) float g_route_logits_scratch[kMaxLogits + 64];
 
 // Device address of g_route_logits_scratch on the current device, or nullptr.
 float* scratch_on_current_device() {
-  static float* cached[128] = {};
+  static std::atomic<float*> cached[128] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-  if (!cached[dev]) {
+  float* s = cached[dev].load(std::memory_order_relaxed);
+  if (!s) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_logits_scratch) != cudaSuccess) return nullptr;
-    cached[dev] = static_cast<float*>(p);
+    s = static_cast<float*>(p);
+    cached[dev].store(s, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return s;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
