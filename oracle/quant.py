@@ -158,7 +158,14 @@ def quantize_nvfp4(w_bits: np.ndarray):
     g float32 [E]).
     """
     assert w_bits.ndim == 3
-    w = bf16_to_f32(w_bits)
+    return quantize_nvfp4_f32(bf16_to_f32(w_bits))
+
+
+def quantize_nvfp4_f32(w: np.ndarray):
+    """The NVFP4 recipe of quantize_nvfp4 on float32 values [E][N][K] (one tensor per
+    leading index); the same steps, for inputs that are not bf16 (activations)."""
+    w = np.asarray(w, dtype=np.float32)
+    assert w.ndim == 3
     E, N, K = w.shape
     amax_t = np.max(np.abs(w.reshape(E, -1)), axis=-1).astype(np.float32)
     g = (amax_t / np.float32(6 * 448)).astype(np.float32)
