@@ -119,6 +119,20 @@ def _p(t: torch.Tensor | None) -> int | None:
     return t.data_ptr()
 
 
+def _check(t: torch.Tensor | None, what: str, dtype=None, numel: int | None = None) -> None:
+    """Caller-provided buffers: the C entry points take plain pointers and cannot check
+    sizes, so the binding checks element type and element count before passing them."""
+    if t is None:
+        return
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{what}: expected {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{what}: needs at least {numel} elements, has {t.numel()}")
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
 def _bits(t: torch.Tensor) -> torch.Tensor:
     """bf16 tensors travel as their 16-bit patterns."""
     if t.dtype == torch.bfloat16:
@@ -135,6 +149,8 @@ def moe_quantize_w4g128(w: torch.Tensor, packed: torch.Tensor | None = None, sca
     E, N, K = w.shape
     packed = torch.empty((E, N, K // 8), dtype=torch.int32, device=w.device) if packed is None else packed
     scales = torch.empty((E, N, K // 128), dtype=torch.bfloat16, device=w.device) if scales is None else scales
+    _check(packed, "packed", (torch.int32, torch.uint32), E * N * (K // 8))
+    _check(scales, "scales", _BF16, E * N * (K // 128))
     _call("moe_quantize_w4g128", _p(_bits(w)), E, N, K, _p(packed), _p(scales), _stream(stream))
     return packed, scales
 
@@ -145,6 +161,8 @@ def moe_pack_bitplanes(w: torch.Tensor, planes: torch.Tensor | None = None, scal
     E, N, K = w.shape
     planes = torch.empty((E, 8, N, K // 32), dtype=torch.int32, device=w.device) if planes is None else planes
     scales = torch.empty((E, N, K // 128), dtype=torch.bfloat16, device=w.device) if scales is None else scales
+    _check(planes, "planes", (torch.int32, torch.uint32), E * 8 * N * (K // 32))
+    _check(scales, "scales", _BF16, E * N * (K // 128))
     _call("moe_pack_bitplanes", _p(_bits(w)), E, N, K, _p(planes), _p(scales), _stream(stream))
     return planes, scales
 
@@ -156,6 +174,9 @@ def moe_quantize_nvfp4(w: torch.Tensor, codes=None, block_scales=None, gscale=No
     block_scales = (torch.empty((E, N, K // 16), dtype=torch.uint8, device=w.device)
                     if block_scales is None else block_scales)
     gscale = torch.empty((E,), dtype=torch.float32, device=w.device) if gscale is None else gscale
+    _check(codes, "codes", torch.uint8, E * N * (K // 2))
+    _check(block_scales, "block_scales", torch.uint8, E * N * (K // 16))
+    _check(gscale, "gscale", torch.float32, E)
     _call("moe_quantize_nvfp4", _p(_bits(w)), E, N, K, _p(codes), _p(block_scales), _p(gscale), _stream(stream))
     return codes, block_scales, gscale
 
@@ -183,6 +204,17 @@ class Routing:
         return RoutingT(_p(self.topk_ids), _p(self.topk_w), _p(self.expert_offsets), _p(self.sorted_pair),
                         _p(self.pair_to_row), _p(self.expert_list))
 
+    def check(self, T: int, E: int, k: int) -> "Routing":
+        """Raises unless the buffers hold a routing of T tokens, E experts, top-k."""
+        P = T * k
+        _check(self.topk_ids, "topk_ids", torch.int32, P)
+        _check(self.topk_w, "topk_w", torch.float32, P)
+        _check(self.expert_offsets, "expert_offsets", torch.int32, E + 1)
+        _check(self.sorted_pair, "sorted_pair", torch.int32, P)
+        _check(self.pair_to_row, "pair_to_row", torch.int32, P)
+        _check(self.expert_list, "expert_list", torch.int32, E + 1)
+        return self
+
 
 def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:
     return int(load().moe_route_workspace_bytes(T, E, k))
@@ -198,7 +230,9 @@ def moe_route_topk(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor |
                    out: Routing | None = None, workspace: torch.Tensor | None = None, stream=None) -> Routing:
     T, H = x.shape
     E = w_router.shape[0]
-    out = Routing.empty(T, E, k, x.device) if out is None else out
+    out = (Routing.empty(T, E, k, x.device) if out is None else out).check(T, E, k)
+    _check(w_router, "w_router", _BF16, E * H)
+    _check(bias, "bias", torch.float32, E)
     if workspace is None:
         workspace = moe_route_workspace(T, E, k, x.device)
     rc = out.c()
@@ -214,7 +248,9 @@ def moe_route_topk_noalloc(x: torch.Tensor, w_router: torch.Tensor, bias: torch.
     by the library.  Calls that overlap on one GPU race on that array."""
     T, H = x.shape
     E = w_router.shape[0]
-    out = Routing.empty(T, E, k, x.device) if out is None else out
+    out = (Routing.empty(T, E, k, x.device) if out is None else out).check(T, E, k)
+    _check(w_router, "w_router", _BF16, E * H)
+    _check(bias, "bias", torch.float32, E)
     rc = out.c()
     _call("moe_route_topk_noalloc", _p(_bits(x)), _p(_bits(w_router)), _p(bias), T, H, E, k, ctypes.byref(rc),
           _stream(stream))
@@ -226,6 +262,8 @@ def moe_select_bits(topk_w: torch.Tensor, k: int, thresholds=(0.05, 0.15, 0.30),
     n = topk_w.numel()
     T = n // k
     bits = torch.empty(max(n, 1), dtype=torch.uint8, device=topk_w.device) if bits is None else bits
+    _check(topk_w, "topk_w", torch.float32)
+    _check(bits, "bits", torch.uint8, n)
     thr = (ctypes.c_float * 3)(*thresholds)
     ch = (ctypes.c_uint8 * 4)(*choices)
     _call("moe_select_bits", _p(topk_w), T, k, thr, ch, _p(bits), _stream(stream))
@@ -239,6 +277,9 @@ def moe_bitplane_distortion(planes: torch.Tensor, scales: torch.Tensor, delta: t
     E, _, N, K32 = planes.shape
     K = K32 * 32
     delta = torch.empty((E, 8, K), dtype=torch.float64, device=planes.device) if delta is None else delta
+    _check(planes, "planes", (torch.int32, torch.uint32))
+    _check(scales, "scales", _BF16, E * N * (K // 128))
+    _check(delta, "delta", torch.float64, E * 8 * K)
     _call("moe_bitplane_distortion", _p(planes), _p(_bits(scales)), E, N, K, _p(delta), _stream(stream))
     return delta
 
@@ -247,6 +288,7 @@ def moe_activation_moments(x: torch.Tensor, m: torch.Tensor | None = None, strea
     """m fp64 [H]: mean over the T tokens of x [T][H] (bf16) squared."""
     T, H = x.shape
     m = torch.empty(H, dtype=torch.float64, device=x.device) if m is None else m
+    _check(m, "m", torch.float64, H)
     _call("moe_activation_moments", _p(_bits(x)), T, H, _p(m), _stream(stream))
     return m
 
@@ -258,6 +300,11 @@ def moe_allocate_bits(delta: torch.Tensor, m: torch.Tensor, expert_offsets: torc
     multiplier is written to ``lam`` (fp64 scalar tensor) when given."""
     E, _, K = delta.shape
     bits_e = torch.empty(E, dtype=torch.uint8, device=delta.device) if bits_e is None else bits_e
+    _check(delta, "delta", torch.float64)
+    _check(m, "m", torch.float64, K)
+    _check(expert_offsets, "expert_offsets", torch.int32, E + 1)
+    _check(bits_e, "bits_e", torch.uint8, E)
+    _check(lam, "lam", torch.float64, 1)
     ch = (ctypes.c_uint8 * len(choices))(*choices)
     _call("moe_allocate_bits", _p(delta), _p(m), _p(expert_offsets), E, K, ch, len(choices), float(budget),
           _p(bits_e), _p(lam), _stream(stream))
@@ -269,6 +316,9 @@ def moe_expand_bits(topk_ids: torch.Tensor, bits_e: torch.Tensor, k: int, bits: 
     """Per-pair widths bits[p] = bits_e[topk_ids[p]] for moe_grouped_ffn."""
     n = topk_ids.numel()
     bits = torch.empty(max(n, 1), dtype=torch.uint8, device=topk_ids.device) if bits is None else bits
+    _check(topk_ids, "topk_ids", torch.int32)
+    _check(bits_e, "bits_e", torch.uint8)
+    _check(bits, "bits", torch.uint8, n)
     _call("moe_expand_bits", _p(topk_ids), _p(bits_e), n // k, k, _p(bits), _stream(stream))
     return bits
 
@@ -303,6 +353,8 @@ def moe_cache_plan(state, need):
     import numpy as np
     need = np.ascontiguousarray(need, dtype=np.uint8)
     E = need.size
+    if state.nbytes < 16 or int(np.asarray(state).view(np.int32)[1]) != E:
+        raise ValueError("need: one entry per expert of the cache state")
     se, ss = np.zeros(E, np.int32), np.zeros(E, np.int32)
     lo, hi = np.zeros(E, np.uint8), np.zeros(E, np.uint8)
     rs = np.zeros(E + 1, np.int32)
@@ -315,6 +367,8 @@ def moe_cache_plan(state, need):
 def moe_cache_slots(state, S: int):
     """(expert_of int32 [S], planes uint8 [S]) of a cache state."""
     import numpy as np
+    if state.nbytes < 16 or int(np.asarray(state).view(np.int32)[2]) != S:
+        raise ValueError("S: the cache state's slot count")
     eo, pl = np.zeros(S, np.int32), np.zeros(S, np.uint8)
     _call("moe_cache_slots", _hp(state), _hp(eo), _hp(pl))
     return eo, pl
@@ -335,6 +389,28 @@ class Experts:
     def c(self) -> ExpertsT:
         return ExpertsT(self.fmt, _p(self.w13), _p(self.w13_scale), _p(self.w2), _p(self.w2_scale),
                         _p(self.w13_gscale), _p(self.w2_gscale))
+
+    def check(self, H: int, I: int, E: int) -> "Experts":
+        """Raises unless the buffers hold E experts of this format for hidden H and
+        intermediate I (sizes as the quantisers write them)."""
+        n13, n2 = 2 * I * H, H * I  # weights per matrix of one expert
+        if self.fmt == FMT_W4G128:
+            sizes = ((self.w13, n13 // 8, (torch.int32, torch.uint32)), (self.w2, n2 // 8, (torch.int32, torch.uint32)),
+                     (self.w13_scale, n13 // 128, _BF16), (self.w2_scale, n2 // 128, _BF16))
+        elif self.fmt == FMT_BITPLANE8:
+            sizes = ((self.w13, n13 // 4, (torch.int32, torch.uint32)), (self.w2, n2 // 4, (torch.int32, torch.uint32)),
+                     (self.w13_scale, n13 // 128, _BF16), (self.w2_scale, n2 // 128, _BF16))
+        elif self.fmt == FMT_NVFP4:
+            sizes = ((self.w13, n13 // 2, torch.uint8), (self.w2, n2 // 2, torch.uint8),
+                     (self.w13_scale, n13 // 16, torch.uint8), (self.w2_scale, n2 // 16, torch.uint8),
+                     (self.w13_gscale, 1, torch.float32), (self.w2_gscale, 1, torch.float32))
+            if self.w13_gscale is None or self.w2_gscale is None:
+                raise ValueError("NVFP4 experts need their per-expert scales")
+        else:
+            raise ValueError(f"unknown format {self.fmt}")
+        for i, (t, per_expert, dt) in enumerate(sizes):
+            _check(t, f"experts buffer {i}", dt, per_expert * E)
+        return self
 
 
 def quantize_experts(fmt: int, w13: torch.Tensor, w2: torch.Tensor, stream=None) -> Experts:
@@ -360,6 +436,10 @@ def moe_grouped_ffn(x: torch.Tensor, routing: Routing, experts: Experts, I: int,
                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     T, H = x.shape
     y_rows = torch.empty((max(T * k, 1), H), dtype=torch.bfloat16, device=x.device) if y_rows is None else y_rows
+    routing.check(T, E, k)
+    experts.check(H, I, E)
+    _check(bits, "bits", torch.uint8, T * k)
+    _check(y_rows, "y_rows", _BF16, T * k * H)
     need = moe_ffn_workspace_bytes(T, H, I, E, k, experts.fmt)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
@@ -373,6 +453,11 @@ def moe_combine(y_rows: torch.Tensor, routing: Routing, T: int, k: int, residual
                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     H = y_rows.shape[1]
     out = torch.empty((T, H), dtype=torch.bfloat16, device=y_rows.device) if out is None else out
+    _check(y_rows, "y_rows", _BF16, T * k * H)
+    _check(routing.topk_w, "topk_w", torch.float32, T * k)
+    _check(routing.pair_to_row, "pair_to_row", torch.int32, T * k)
+    _check(residual, "residual", _BF16, T * H)
+    _check(out, "out", _BF16, T * H)
     rc = routing.c()
     _call("moe_combine", _p(y_rows), ctypes.byref(rc), _p(residual), T, H, k, _p(out), _stream(stream))
     return out

@@ -1,6 +1,8 @@
 """The library's slot-cache planner (host entry points, no GPU) against the oracle:
 every step's service order, slots, fetched plane ranges and rounds, and the slots'
 contents after it, on seeded routing sequences; plus argument validation."""
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -73,5 +75,13 @@ def test_cache_validation(lib):
         moe.moe_cache_plan(state, np.array([4, 0, 0, 0], np.uint8))  # above the planes
     eo, pl = moe.moe_cache_slots(state, 2)
     assert eo.tolist() == [-1, -1] and pl.tolist() == [0, 0]        # untouched by the rejected call
-    with pytest.raises(moe.MoeError):
-        moe.moe_cache_plan(np.zeros(8, np.int64), np.zeros(4, np.uint8))  # not an initialised state
+    raw = np.zeros(8, np.int64)  # not an initialised state: the library rejects it
+    outs = [np.zeros(4, np.int32), np.zeros(4, np.int32), np.zeros(4, np.uint8), np.zeros(4, np.uint8),
+            np.zeros(5, np.int32)]
+    nr = ctypes.c_int32(0)
+    assert lib.moe_cache_plan(raw.ctypes.data, np.zeros(4, np.uint8).ctypes.data,
+                              *[o.ctypes.data for o in outs], ctypes.byref(nr)) == 1
+    with pytest.raises(ValueError):  # the binding checks need against the state's expert count
+        moe.moe_cache_plan(state, np.zeros(5, np.uint8))
+    with pytest.raises(ValueError):
+        moe.moe_cache_slots(state, 3)
