@@ -312,7 +312,12 @@ size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64
  * gathered into routed order; contents need not be initialised).  Not bit-exact: fp32
  * accumulation order, the rounding of h (and, on the GEMM path, of each dequantised
  * W4 weight to bf16) differ from an fp64 reference (ExactMoE: the low-bit layer is
- * not numerically identical to BF16); the FFN tolerance covers both paths. */
+ * not numerically identical to BF16); the FFN tolerance covers both paths.
+ * Range: the GEMV stages W4 activations as fp16 x/16 and x/256, and NVFP4 activations
+ * and h (both paths) as fp16 * 2^-8, so |x| < 2^20 (W4) and |x|, |h| < 2^24 (NVFP4) keep
+ * them finite; magnitudes below 2^-10 (W4) or 2^-6 (NVFP4) fall into fp16's subnormal
+ * range (absolute error at most 2^-20 or 2^-16).  Bitplane activations are staged in
+ * bf16 scaled by up to 2^7 (|x| < 2^120). */
 moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
                              const moe_experts_t* experts, const uint8_t* bits,
                              int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
