@@ -61,11 +61,17 @@ PREFILL = {
                                           "per 16, fp32 per tensor), U(-0.02, 0.02) bf16 router, 4096 fresh "
                                           "tokens per step"),
     "bitplane-h2048-e64": dict(T=64, H=2048, I=1024, E=64, k=8, router="normal", zipf=False, seed=0x5EED0004,
-                               fmt="bitplane", budget=3.0, choices=(2, 3, 4, 8), profile_tokens=2048,
-                               desc="one MoE FFN layer, H2048 I1024 E64 top-8, 8-bitplane experts read at "
-                                    "per-expert widths from a budgeted allocation (3.0 bits per weight of "
-                                    "routing-weighted reads over {2,3,4,8}, profiled on 2048 tokens), bf16 "
-                                    "router, 64 fresh tokens per step"),
+                               fmt="bitplane", bits="rule",
+                               desc="one MoE FFN layer, H2048 I1024 E64 top-8, 8-bitplane experts, each "
+                                    "(token, expert) read at b in {2,3,4,8} planes by routing-score thresholds "
+                                    "{0.05,0.15,0.3}, bf16 router, 64 fresh tokens per step"),
+    "bitplane-h2048-e64-duorate": dict(T=64, H=2048, I=1024, E=64, k=8, router="normal", zipf=False,
+                                       seed=0x5EED0004, fmt="bitplane", bits="allocated", budget=3.0,
+                                       choices=(2, 3, 4, 8), profile_tokens=2048,
+                                       desc="one MoE FFN layer, H2048 I1024 E64 top-8, 8-bitplane experts read at "
+                                            "per-expert widths from a budgeted allocation (3.0 bits per weight of "
+                                            "routing-weighted reads over {2,3,4,8}, profiled on 2048 tokens), "
+                                            "bf16 router, 64 fresh tokens per step"),
 }
 # bitplane experts: bytes of one plane of one expert's w13 + w2, and of their bf16 scales
 BP_PLANE_BYTES = (2 * I * H + H * I) // 8
@@ -86,7 +92,7 @@ def parse_args(argv=None):
                     help="layers in the stack (16 is the benchmark workload; fewer only for profiling)")
     args = ap.parse_args(argv)
     if args.steps is None:
-        args.steps = 512 if args.workload in ("decode", "bitplane-h2048-e64") else 20
+        args.steps = 512 if args.workload == "decode" or args.workload.startswith("bitplane") else 20
     return args
 
 
@@ -502,7 +508,10 @@ class PrefillLayer:
         moe, c = self.moe, self.cfg
         moe.moe_route_topk(self.x, self.wr, self.bias, c["k"], out=self.routing, workspace=self.route_ws)
         if self.bits is not None:
-            moe.moe_expand_bits(self.routing.topk_ids, self.bits_e, c["k"], bits=self.bits)
+            if c["bits"] == "rule":  # b from the routing weights by thresholds (0.05, 0.15, 0.3)
+                moe.moe_select_bits(self.routing.topk_w, c["k"], bits=self.bits)
+            else:  # per-expert widths of the budgeted allocation
+                moe.moe_expand_bits(self.routing.topk_ids, self.bits_e, c["k"], bits=self.bits)
         if self.ffn_events is not None:
             self.ffn_events[0].record()
         moe.moe_grouped_ffn(self.x, self.routing, self.copies[copy], c["I"], c["E"], c["k"], y_rows=self.y_rows,
@@ -532,7 +541,7 @@ def run_prefill(args, rank, world, local):
     K, W = args.steps, max(args.warmup, 3)
     layer = PrefillLayer(moe, torch, device, cfg)
     allocation = layer.allocate_widths(torch, device, rank_seed(cfg["seed"], rank)) \
-        if layer.fmt == moe.FMT_BITPLANE8 else None
+        if cfg.get("bits") == "allocated" else None
     inputs = torch.empty((W + K, T, Hh), dtype=torch.bfloat16, device=device)
     moe.moe_synth_normal_bf16(inputs, rank_seed(cfg["seed"], rank) + synth.SEED_X, 1.0)
     torch.cuda.synchronize()
@@ -601,23 +610,31 @@ def run_prefill(args, rank, world, local):
                 layer.step(c_)
     torch.cuda.current_stream().wait_stream(cap)
     ffn_ms, ffn_bytes = [], []
-    bits_e = layer.bits_e.cpu().to(torch.int64) if layer.bits_e is not None else None
+    bitplane = layer.bits is not None
     for s in range(W, W + min(K, 10)):
         layer.x.copy_(inputs[s])
         g2s[s % nc].replay()
         torch.cuda.synchronize()
         ffn_ms.append(layer.ffn_events[0].elapsed_time(layer.ffn_events[1]))
-        if bits_e is not None:
-            # the weight stream of this step: each routed expert's prefix of b_e planes, once
-            routed = torch.diff(layer.routing.expert_offsets.to(torch.int64)).cpu() > 0
-            ffn_bytes.append(int((bits_e[routed] * BP_PLANE_BYTES + BP_SCALE_BYTES).sum()))
+        if bitplane:
+            # the weight stream of this step: each routed expert's prefix of b_max planes (the
+            # widest of its pairs), once, with its scales
+            offs = layer.routing.expert_offsets.cpu().tolist()
+            sp = layer.routing.sorted_pair.cpu().tolist()
+            bits = layer.bits.cpu().tolist()
+            nbytes = 0
+            for e in range(Ee):
+                if offs[e + 1] > offs[e]:
+                    bmax = max(bits[sp[r]] for r in range(offs[e], offs[e + 1]))
+                    nbytes += bmax * BP_PLANE_BYTES + BP_SCALE_BYTES
+            ffn_bytes.append(nbytes)
     layer.ffn_events = None
     hbm, bf16_peak, peak_kind = measured_peaks()
     avg_s = statistics.mean(ffn_ms) / 1e3
-    if bits_e is not None:
+    if bitplane:
         achieved = sum(ffn_bytes) / (sum(ffn_ms) / 1e3) / 1e9
-        tr = committed_traffic("traffic_bitplane.json")
-        # DRAM bytes of one captured call (all 64 experts at 3 planes, as this workload allocates)
+        tr = committed_traffic("traffic_bitplane.json") if allocation is not None else None
+        # DRAM bytes of one captured call (all 64 experts at 3 planes, as the allocated workload reads)
         traffic = tr["dram_bytes_per_call"] if tr else None
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(achieved / hbm, 4), "peak_kind": peak_kind + " HBM copy", "traffic": traffic,
@@ -643,7 +660,7 @@ def run_prefill(args, rank, world, local):
             "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,
                        "top_k": k, "parallelism": f"dp{world} (independent replicas)",
                        "l2": ("no flush: each step reads more than %.1f GB of expert weights, > 126 MB L2"
-                              % (Ee * 3 * Hh * Ii / 2 / 1e9)) if allocation is None else
+                              % (Ee * 3 * Hh * Ii / 2 / 1e9)) if not bitplane else
                              ("no flush: each step reads about %.0f MB of expert planes and scales, and "
                               "steps rotate over 4 device copies of the weights (> 126 MB L2 between "
                               "reuses)" % (statistics.mean(ffn_bytes) / 1e6))},
@@ -707,7 +724,7 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
     else:
         ex = Experts(FMT_BITPLANE8 if bitplane else FMT_W4G128, w13q, w13s, w2q, w2s)
     t0 = time.perf_counter()
-    if bitplane:
+    if bitplane and cfg.get("bits") == "allocated":
         # the same per-step path at per-expert widths (every expert at 3 planes, the budget's mean)
         r = route(x, wr, bias, k, Ee)
         y = grouped_ffn(x, r.offsets, r.sorted_pair, k, ex, expand_bits(r.ids, np.full(Ee, 3, np.uint8)))
@@ -776,7 +793,8 @@ def cpu_baseline_prefill(cfg, seed: int):
     v, secs, thr = oracle_prefill_sample(cfg, n, seed)
     return {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
             "sample": f"{n} tokens through the layer ({secs:.1f} s of CPU work: routing, dequantisation of "
-                      f"their experts" + (" at 3 planes each" if cfg.get("fmt") == "bitplane" else "")
+                      f"their experts" + (" at 3 planes each" if cfg.get("bits") == "allocated" else
+                                          " at the thresholds' widths" if cfg.get("fmt") == "bitplane" else "")
                       + ", SwiGLU, combine); weights generated and quantised untimed"}
 
 
