@@ -21,18 +21,24 @@
  *               compensation quantisation; bit-width per expert from routing scores.
  *   [MoET]      "MoET in FP4 MoE Inference" (Q&A page), answer and references:
  *               FP4/INT4 expert weights, router at higher precision, NVFP4.
+ *   [DuoRate]   "DuoRate: Two-Rate Per-Expert Precision Allocation for Mixture-of-
+ *               Experts Serving", key concepts: a resident and a routing-weighted
+ *               read rate; a distortion tensor baked offline, unlabeled profiling,
+ *               one dot product per expert and a bisection to a read budget.
  *
  * Conventions shared by every entry point
  *   - bf16 values are passed as uint16_t bit patterns.
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise, owned
  *     by the caller; the library never allocates, frees or keeps a pointer after
- *     the call returns.  Device pointers must be 16-byte aligned.
+ *     the call returns.  Device pointers must be 16-byte aligned unless a call
+ *     states a smaller alignment.
  *   - Every call only enqueues work on `stream` (a cudaStream_t; NULL means the
  *     legacy default stream) and returns without synchronising.
  *   - All arguments are validated on the host before anything is launched; an
  *     invalid call launches nothing and returns an error code.  A failed launch
  *     returns MOE_ERR_CUDA.  No C++ exception crosses the ABI.
- *   - T = 0 (no tokens) is valid and launches nothing.
+ *   - T = 0 (no tokens) is valid and launches nothing, except where a call
+ *     requires T >= 1 (the activation moments).
  *   - Shapes: weights are row-major [E][N][K] with K contiguous.  The gate/up
  *     matrix w13 of expert e is [2I][H] (rows 0..I-1 gate, I..2I-1 up); the down
  *     matrix w2 is [H][I].
