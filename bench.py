@@ -88,6 +88,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cache-slots", type=int, default=0,
+                    help="decode with each layer's experts in pinned host memory and this many device slots "
+                         "per layer (0: every expert resident in HBM)")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers in the stack (16 is the benchmark workload; fewer only for profiling)")
     args = ap.parse_args(argv)
@@ -270,6 +273,90 @@ class DecodeStack:
         return self.L * (route + 3)
 
 
+class CachedDecodeStack(DecodeStack):
+    """The decode stack with every layer's experts in pinned host memory and S device
+    slots per layer: route, plan the step on the device, permute the pairs by slot, fetch
+    the missing experts over the host link, FFN on the slots, combine."""
+
+    def __init__(self, moe, torch, device, batch: int, seed: int, layers: int, slots: int):
+        super().__init__(moe, torch, device, batch, seed, layers)
+        S, B = slots, batch
+        self.S = S
+        pin = lambda t: t.cpu().pin_memory()
+        zeros = lambda t: torch.zeros((S,) + tuple(t.shape[1:]), dtype=t.dtype, device=device)
+        self.host, self.slots, self.states, self.plans = [], [], [], []
+        for l in range(layers):
+            wr, ex = self.layers[l]
+            self.host.append(moe.Experts(ex.fmt, pin(ex.w13), pin(ex.w13_scale), pin(ex.w2), pin(ex.w2_scale)))
+            self.slots.append(moe.Experts(ex.fmt, zeros(ex.w13), zeros(ex.w13_scale), zeros(ex.w2),
+                                          zeros(ex.w2_scale)))
+            self.states.append(moe.moe_cache_state_device(E, S, 1, device))
+            self.plans.append(moe.CachePlan.empty(E, device))
+            self.layers[l] = (wr, None)  # the device copy of the experts is dropped
+        torch.cuda.empty_cache()
+        i32 = dict(dtype=torch.int32, device=device)
+        self.slot_ids = torch.empty(B * K_TOP, **i32)
+        self.rs = moe.Routing(self.slot_ids, self.routing.topk_w, torch.empty(S + 1, **i32),
+                              torch.empty(B * K_TOP, **i32), torch.empty(B * K_TOP, **i32), torch.empty(S + 1, **i32))
+        self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(B, H, I, S, K_TOP, moe.FMT_W4G128), 16),
+                                  dtype=torch.uint8, device=device)
+        self.fetch_events = None
+
+    def layer(self, l, log_active=False):
+        moe = self.moe
+        wr, _ = self.layers[l]
+        x, nxt = self.xs[l], self.xs[l + 1]
+        moe.moe_route_topk(x, wr, None, K_TOP, out=self.routing, workspace=self.route_ws)
+        moe.moe_cache_step(self.states[l], E, self.S, self.routing, self.B, K_TOP, slot_ids=self.slot_ids,
+                           plan=self.plans[l])
+        moe.moe_permute(self.slot_ids, self.B, K_TOP, self.S, out=self.rs)
+        if self.fetch_events is not None:
+            self.fetch_events[l][0].record()
+        moe.moe_cache_fetch(self.plans[l], E, self.host[l], self.slots[l], H, I)
+        if self.fetch_events is not None:
+            self.fetch_events[l][1].record()
+        moe.moe_grouped_ffn(x, self.rs, self.slots[l], I, self.S, K_TOP, y_rows=self.y_rows, workspace=self.ffn_ws)
+        moe.moe_combine(self.y_rows, self.rs, self.B, K_TOP, residual=x, out=nxt)
+        if log_active:
+            self.n_active[l:l + 1].copy_(self.routing.expert_list[:1])
+
+    def fetched(self):
+        """(bytes copied over the host link, experts served, hits) of the last step, all layers."""
+        total = served = hits = 0
+        for plan in self.plans:
+            n = int(plan.nserved.item())
+            lo = plan.fetch_lo[:n].cpu().tolist()
+            hi = plan.fetch_hi[:n].cpu().tolist()
+            total += sum(W4_EXPERT_BYTES for a, b in zip(lo, hi) if b > a)
+            served += n
+            hits += sum(1 for a, b in zip(lo, hi) if a == b)
+        return total, served, hits
+
+    @property
+    def kernels_per_step(self):
+        # router, cache step, permutation by slot, fetch (w13, w2), gate/up, down, combine
+        route = 1 if (self.B <= 16 and self.B * H * 2 <= 64 * 1024) else 3
+        return self.L * (route + 7)
+
+
+def measured_h2d_gbs(torch, device, nbytes: int = 256 << 20) -> float:
+    """Pinned host -> device copy bandwidth (median of 5 copies of 256 MB), the peak of the
+    host link the slot cache reads over."""
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / 1e3)
+    return nbytes / statistics.median(ts) / 1e9
+
+
 def run_gpu(args, rank, world, local):
     import torch
     torch.cuda.set_device(local)
@@ -282,7 +369,12 @@ def run_gpu(args, rank, world, local):
     B, K, W = args.batch, args.steps, max(args.warmup, 3)
     seed = rank_seed(SEED_BASE, rank)
     L = args.layers
-    stack = DecodeStack(moe, torch, device, B, seed, L)
+    if args.cache_slots:
+        if not (1 <= args.cache_slots <= E and args.cache_slots >= min(E, B * K_TOP)):
+            raise SystemExit("--cache-slots must be in [min(E, batch * top-k), E]")
+        stack = CachedDecodeStack(moe, torch, device, B, seed, L, args.cache_slots)
+    else:
+        stack = DecodeStack(moe, torch, device, B, seed, L)
     # a fresh seeded N(0,1) batch for every step (warm-up and timed), resident in HBM
     n_steps = W + K
     inputs = torch.empty((n_steps, B, H), dtype=torch.bfloat16, device=device)
@@ -350,10 +442,72 @@ def run_gpu(args, rank, world, local):
         e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": B * H * 2,
                "d2h_bytes_per_step": B * H * 2}
 
+    if args.cache_slots:
+        roofline, act = cached_roofline(torch, device, stack, cap, inputs, W, K)
+    else:
+        roofline, act = resident_roofline(torch, stack, cap, inputs, W, K, B)
+    result = None
+    if rank == 0:
+        cfg_extra = {} if not args.cache_slots else {
+            "cache": "experts of each layer in pinned host memory, %d device slots per layer, planned on the "
+                     "device each step, missing experts read over the host link" % args.cache_slots}
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, "
+                                                          "N(0,0.02) bf16 weights quantised to W4A16 g128)",
+            "config": dict({"workload": "decode stack: %d chained OLMoE-like MoE FFN layers (H2048 I1024 E64 "
+                                        "top-8, W4A16 g128 experts, bf16 router), residual add, batch %d "
+                                        "tokens/step" % (L, B),
+                            "layers": L, "batch": B, "hidden": H, "intermediate": I, "experts": E, "top_k": K_TOP,
+                            "parallelism": f"dp{world} (independent replicas)",
+                            "l2": "no flush: each step streams ~%.1f GB of distinct expert weights, > 126 MB L2"
+                                  % (statistics.mean(act) * W4_EXPERT_BYTES * L / 1e9)}, **cfg_extra),
+            "gpu_launches": stack.kernels_per_step * K,
+            "clocks": clk, "roofline": roofline, "e2e": e2e,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        del graph
+        dist.destroy_process_group()
+    return result
+
+
+def cached_roofline(torch, device, stack, cap, inputs, W, K):
+    """The fetch (moe_cache_fetch, both launches) against the measured pinned host ->
+    device bandwidth: bytes copied over the host link per call / its event-timed duration."""
+    stack.fetch_events = [(torch.cuda.Event(enable_timing=True, external=True),
+                           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(stack.L)]
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g2, stream=cap):
+            stack.step(log_active=True)
+    torch.cuda.current_stream().wait_stream(cap)
+    ms, nbytes, served, hits, act = 0.0, 0, 0, 0, []
+    for s in range(W, W + min(K, 32)):
+        stack.xs[0].copy_(inputs[s])
+        g2.replay()
+        torch.cuda.synchronize()
+        ms += sum(a.elapsed_time(b) for a, b in stack.fetch_events)
+        b_, n_, h_ = stack.fetched()
+        nbytes, served, hits = nbytes + b_, served + n_, hits + h_
+        act += stack.n_active.cpu().tolist()
+    stack.fetch_events = None
+    del g2
+    peak = measured_h2d_gbs(torch, device)
+    achieved = nbytes / (ms / 1e3) / 1e9 if ms > 0 else 0.0
+    return ({"bound": "host-link", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "GB/s",
+             "frac": round(achieved / peak, 4), "peak_kind": "measured pinned host->device copy in this run",
+             "traffic": None, "kernel": "k_cache_fetch (w13 + w2 of the missing experts, one moe_cache_fetch call)",
+             "fetched_bytes_per_step": round(nbytes / min(K, 32)),
+             "hit_rate": round(hits / served, 4) if served else None}, act)
+
+
+def resident_roofline(torch, stack, cap, inputs, W, K, B):
     # ---- roofline of the dominant op: the grouped W4 GEMV (gate/up + down launches of
     # moe_grouped_ffn), timed with CUDA events recorded on its stream inside a graph
     stack.ffn_events = [(torch.cuda.Event(enable_timing=True, external=True),
-                         torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
+                         torch.cuda.Event(enable_timing=True, external=True)) for _ in range(stack.L)]
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.stream(cap):
         with torch.cuda.graph(g2, stream=cap):
@@ -380,28 +534,8 @@ def run_gpu(args, rank, world, local):
                 "kernel": "k_ffn_gemv<W4> gate/up + down (one moe_grouped_ffn call)",
                 "algorithmic_bytes_per_call": round(algo_bytes), "avg_call_us": round(avg_ffn_s * 1e6, 2),
                 "distinct_experts_per_layer": round(statistics.mean(act), 2)}
-
-    result = None
-    if rank == 0:
-        result = {
-            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, "
-                                                          "N(0,0.02) bf16 weights quantised to W4A16 g128)",
-            "config": {"workload": "decode stack: %d chained OLMoE-like MoE FFN layers (H2048 I1024 E64 top-8, "
-                                   "W4A16 g128 experts, bf16 router), residual add, batch %d tokens/step" % (L, B),
-                       "layers": L, "batch": B, "hidden": H, "intermediate": I, "experts": E, "top_k": K_TOP,
-                       "parallelism": f"dp{world} (independent replicas)",
-                       "l2": "no flush: each step streams ~%.1f GB of distinct expert weights, > 126 MB L2"
-                             % (statistics.mean(act) * W4_EXPERT_BYTES * L / 1e9)},
-            "gpu_launches": stack.kernels_per_step * K,
-            "clocks": clk, "roofline": roofline, "e2e": e2e,
-        }
-    if world > 1:
-        import torch.distributed as dist
-        del graph, g2
-        dist.destroy_process_group()
-    return result
+    del g2
+    return roofline, act
 
 
 # ---------------------------------------------------------------- prefill workloads

@@ -43,6 +43,11 @@ class ExpertsT(ctypes.Structure):
                 ("w2_gscale", ctypes.c_void_p)]
 
 
+class CachePlanT(ctypes.Structure):
+    _fields_ = [("served_expert", ctypes.c_void_p), ("served_slot", ctypes.c_void_p), ("fetch_lo", ctypes.c_void_p),
+                ("fetch_hi", ctypes.c_void_p), ("nserved", ctypes.c_void_p), ("overflow", ctypes.c_void_p)]
+
+
 _lib = None
 _vp, _i64, _sz, _u64, _d = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_double
 
@@ -68,10 +73,17 @@ _SIGS = {
     "moe_cache_init": ([_vp, _sz, _i64, _i64, _i64], ctypes.c_int),
     "moe_cache_plan": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
     "moe_cache_slots": ([_vp, _vp, _vp], ctypes.c_int),
+    "moe_cache_step": ([_vp, _i64, _i64, ctypes.POINTER(RoutingT), _vp, _i64, _i64, _vp, ctypes.POINTER(CachePlanT),
+                        _vp], ctypes.c_int),
+    "moe_cache_fetch": ([ctypes.POINTER(CachePlanT), _i64, ctypes.POINTER(ExpertsT), ctypes.POINTER(ExpertsT), _i64,
+                         _i64, _vp], ctypes.c_int),
+    "moe_permute": ([_vp, _i64, _i64, _i64, ctypes.POINTER(RoutingT), _vp], ctypes.c_int),
     "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
     "moe_grouped_ffn": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
                          _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_combine": ([_vp, ctypes.POINTER(RoutingT), _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
+    "moe_gather_rows": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
+    "moe_ids_from_counts": ([_vp, _i64, _i64, _vp, _vp], ctypes.c_int),
     "moe_check_device_errors": ([_vp], ctypes.c_int),
     "moe_synth_normal_bf16": ([_vp, _i64, _i64, _u64, _d, _vp], ctypes.c_int),
     "moe_synth_uniform_bf16": ([_vp, _i64, _i64, _u64, _d, _d, _vp], ctypes.c_int),
@@ -221,8 +233,9 @@ def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:
 
 
 def moe_route_workspace(T: int, E: int, k: int, device) -> torch.Tensor:
-    """A zero-filled router workspace for up to (T, E, k); reusable across calls
-    (each call leaves its completion counter at zero)."""
+    """A zero-filled router workspace for up to (T, E, k): it serves any later call with
+    T' <= T and E' <= E, in any order (the completion counter sits in its first 256
+    bytes whatever the shape, and each call leaves it at zero)."""
     return torch.zeros(max(moe_route_workspace_bytes(T, E, k), 16), dtype=torch.uint8, device=device)
 
 
@@ -412,6 +425,81 @@ class Experts:
             _check(t, f"experts buffer {i}", dt, per_expert * E)
         return self
 
+    def c_host(self) -> ExpertsT:
+        """The same struct over page-locked host tensors (a slot cache's expert store)."""
+        return ExpertsT(self.fmt, _pinned(self.w13), _pinned(self.w13_scale), _pinned(self.w2),
+                        _pinned(self.w2_scale), _pinned(self.w13_gscale), _pinned(self.w2_gscale))
+
+
+def _pinned(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+        raise ValueError("expected a contiguous page-locked host tensor")
+    return t.data_ptr()
+
+
+# ---------------------------------------------------------------- expert slot cache (device)
+@dataclass
+class CachePlan:
+    """Device buffers of one step's cache plan (moe_cache_plan_t)."""
+    served_expert: torch.Tensor
+    served_slot: torch.Tensor
+    fetch_lo: torch.Tensor
+    fetch_hi: torch.Tensor
+    nserved: torch.Tensor
+    overflow: torch.Tensor
+
+    @staticmethod
+    def empty(E: int, device="cuda") -> "CachePlan":
+        i32, u8 = dict(dtype=torch.int32, device=device), dict(dtype=torch.uint8, device=device)
+        return CachePlan(torch.empty(E, **i32), torch.empty(E, **i32), torch.empty(E, **u8), torch.empty(E, **u8),
+                         torch.zeros(1, **i32), torch.zeros(1, **i32))
+
+    def c(self) -> CachePlanT:
+        return CachePlanT(_p(self.served_expert), _p(self.served_slot), _p(self.fetch_lo), _p(self.fetch_hi),
+                          _p(self.nserved), _p(self.overflow))
+
+
+def moe_cache_state_device(E: int, S: int, planes: int, device="cuda") -> torch.Tensor:
+    """A fresh cache state (moe_cache_init on the host) copied to device memory."""
+    host = moe_cache_init(E, S, planes)
+    return torch.from_numpy(host.view("uint8")).to(device)
+
+
+def moe_cache_step(state: torch.Tensor, E: int, S: int, routing: Routing, T: int, k: int,
+                   bits: torch.Tensor | None = None, slot_ids: torch.Tensor | None = None,
+                   plan: CachePlan | None = None, stream=None):
+    """One step's plan on the device; returns (slot_ids int32 [T*k], plan)."""
+    slot_ids = torch.empty(max(T * k, 1), dtype=torch.int32, device=state.device) if slot_ids is None else slot_ids
+    plan = CachePlan.empty(E, state.device) if plan is None else plan
+    routing.check(T, E, k)
+    _check(bits, "bits", torch.uint8, T * k)
+    _check(slot_ids, "slot_ids", torch.int32, T * k)
+    for name in ("served_expert", "served_slot", "fetch_lo", "fetch_hi"):
+        _check(getattr(plan, name), name, None, E)
+    _check(state, "state", torch.uint8, moe_cache_state_bytes(E, S))
+    rc, pc = routing.c(), plan.c()
+    _call("moe_cache_step", _p(state), E, S, ctypes.byref(rc), _p(bits), T, k, _p(slot_ids), ctypes.byref(pc),
+          _stream(stream))
+    return slot_ids, plan
+
+
+def moe_cache_fetch(plan: CachePlan, E: int, host_store: "Experts", slots: "Experts", H: int, I: int, stream=None):
+    host_store.check(H, I, E)
+    slots.check(H, I, int(slots.w13.shape[0]))
+    pc, hc, sc = plan.c(), host_store.c_host(), slots.c()
+    _call("moe_cache_fetch", ctypes.byref(pc), E, ctypes.byref(hc), ctypes.byref(sc), H, I, _stream(stream))
+
+
+def moe_permute(ids: torch.Tensor, T: int, k: int, E: int, out: Routing | None = None, stream=None) -> Routing:
+    """The permutation alone; out.topk_ids and out.topk_w are the caller's (not written)."""
+    out = (Routing.empty(T, E, k, ids.device) if out is None else out).check(T, E, k)
+    _check(ids, "ids", torch.int32, T * k)
+    rc = out.c()
+    _call("moe_permute", _p(ids), T, k, E, ctypes.byref(rc), _stream(stream))
+    return out
+
 
 def quantize_experts(fmt: int, w13: torch.Tensor, w2: torch.Tensor, stream=None) -> Experts:
     """Quantise bf16 w13 [E][2I][H] and w2 [E][H][I] into one of the three formats."""
@@ -461,6 +549,29 @@ def moe_combine(y_rows: torch.Tensor, routing: Routing, T: int, k: int, residual
     rc = routing.c()
     _call("moe_combine", _p(y_rows), ctypes.byref(rc), _p(residual), T, H, k, _p(out), _stream(stream))
     return out
+
+
+def moe_gather_rows(src: torch.Tensor, idx: torch.Tensor, div: int = 1, n: int | None = None,
+                    dst: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dst[i] = src[idx[i] // div] (bf16 rows) for the first n indices."""
+    n = idx.numel() if n is None else n
+    H = src.shape[1]
+    dst = torch.empty((max(n, 1), H), dtype=src.dtype, device=src.device) if dst is None else dst
+    _check(src, "src", _BF16)
+    _check(idx, "idx", torch.int32, n)
+    _check(dst, "dst", _BF16, n * H)
+    _call("moe_gather_rows", _p(_bits(src)), _p(idx), n, div, H, _p(_bits(dst)), _stream(stream))
+    return dst
+
+
+def moe_ids_from_counts(counts: torch.Tensor, n: int, ids: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """ids int32 [n] of received rows from counts int32 [S][El] (n = counts.sum())."""
+    S, El = counts.shape
+    ids = torch.empty(max(n, 1), dtype=torch.int32, device=counts.device) if ids is None else ids
+    _check(counts, "counts", torch.int32, S * El)
+    _check(ids, "ids", torch.int32, n)
+    _call("moe_ids_from_counts", _p(counts), S, El, _p(ids), _stream(stream))
+    return ids
 
 
 def moe_check_device_errors(stream=None) -> None:

@@ -130,7 +130,7 @@ moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const f
   if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned16(bias))) return MOE_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < moe::route_workspace_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MOE_ERR_MISALIGNED;
-  return from_cuda(moe::launch_route(x, w_router, bias, int(T), int(H), int(E), int(k), *out, workspace,
+  return from_cuda(moe::launch_route_ws(x, w_router, bias, int(T), int(H), int(E), int(k), *out, workspace,
                                      as_stream(stream)));
 }
 
@@ -227,6 +227,56 @@ moe_status_t moe_cache_slots(const void* state, int32_t* expert_of, uint8_t* pla
   return MOE_OK;
 }
 
+moe_status_t moe_cache_step(void* state, int64_t E, int64_t S, const moe_routing_t* routing, const uint8_t* bits,
+                            int64_t T, int64_t k, int32_t* slot_ids, const moe_cache_plan_t* plan,
+                            moe_stream_t stream) {
+  if (!state || !routing || !slot_ids || !plan) return MOE_ERR_INVALID_ARG;
+  if (!plan->served_expert || !plan->served_slot || !plan->fetch_lo || !plan->fetch_hi || !plan->nserved ||
+      !plan->overflow)
+    return MOE_ERR_INVALID_ARG;
+  const moe_status_t rs = check_route_shape(T, E, k);
+  if (rs != MOE_OK) return rs;
+  if (S < 1 || S > E) return MOE_ERR_INVALID_ARG;
+  if (S < (T * k < E ? T * k : E)) return MOE_ERR_UNSUPPORTED_SHAPE;  // one round only
+  const moe_status_t rc = check_routing(routing);
+  if (rc != MOE_OK) return rc;
+  if ((reinterpret_cast<uintptr_t>(state) & 7u) || (reinterpret_cast<uintptr_t>(slot_ids) & 3u))
+    return MOE_ERR_MISALIGNED;
+  if (T == 0) return MOE_OK;
+  return from_cuda(moe::launch_cache_step(state, *routing, bits, int(T * k), slot_ids, *plan, as_stream(stream)));
+}
+
+moe_status_t moe_cache_fetch(const moe_cache_plan_t* plan, int64_t E, const moe_experts_t* host_store,
+                             const moe_experts_t* slots, int64_t H, int64_t I, moe_stream_t stream) {
+  if (!plan || !host_store || !slots) return MOE_ERR_INVALID_ARG;
+  if (host_store->fmt != slots->fmt) return MOE_ERR_INVALID_ARG;
+  const void* ps[] = {host_store->w13, host_store->w13_scale, host_store->w2, host_store->w2_scale,
+                      slots->w13, slots->w13_scale, slots->w2, slots->w2_scale};
+  for (const void* p : ps)
+    if (!p) return MOE_ERR_INVALID_ARG;
+  if (host_store->fmt == MOE_FMT_NVFP4 &&
+      (!host_store->w13_gscale || !host_store->w2_gscale || !slots->w13_gscale || !slots->w2_gscale))
+    return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > MOE_MAX_EXPERTS || H % 256 != 0 || I % 128 != 0 || H < 256 || I < 128)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  for (const void* p : ps)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_cache_fetch(*plan, int(E), *host_store, *slots, int(H), int(I), as_stream(stream)));
+}
+
+moe_status_t moe_permute(const int32_t* ids, int64_t T, int64_t k, int64_t E, const moe_routing_t* out,
+                         moe_stream_t stream) {
+  const moe_status_t rs = check_route_shape(T, E, k);
+  if (rs != MOE_OK) return rs;
+  if (!ids || !out || !out->expert_offsets || !out->sorted_pair || !out->pair_to_row || !out->expert_list)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ids) || !aligned16(out->expert_offsets) || !aligned16(out->sorted_pair) ||
+      !aligned16(out->pair_to_row) || !aligned16(out->expert_list))
+    return MOE_ERR_MISALIGNED;
+  if (T == 0) return MOE_OK;  // as moe_route_topk: nothing to permute, no pointer is read
+  return from_cuda(moe::launch_permute(ids, int(T * k), int(E), *out, as_stream(stream)));
+}
+
 moe_status_t moe_select_bits(const float* topk_w, int64_t T, int64_t k, const float thresholds[3],
                              const uint8_t choices[4], uint8_t* bits, moe_stream_t stream) {
   if (!topk_w || !thresholds || !choices || !bits) return MOE_ERR_INVALID_ARG;
@@ -286,6 +336,23 @@ moe_status_t moe_combine(const uint16_t* y_rows, const moe_routing_t* routing, c
   if (s != MOE_OK) return s;
   if (!aligned16(y_rows) || !aligned16(out) || (residual && !aligned16(residual))) return MOE_ERR_MISALIGNED;
   return from_cuda(moe::launch_combine(y_rows, *routing, residual, int(T), int(H), int(k), out, as_stream(stream)));
+}
+
+moe_status_t moe_gather_rows(const uint16_t* src, const int32_t* idx, int64_t n, int64_t div, int64_t H,
+                             uint16_t* dst, moe_stream_t stream) {
+  if (n < 0 || div < 1 || H < 8) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0 || n > INT_MAX || H > INT_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return MOE_OK;
+  if (!src || !idx || !dst) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(idx) & 3u)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_gather_rows_by(src, idx, int(n), int(div), int(H), dst, as_stream(stream)));
+}
+
+moe_status_t moe_ids_from_counts(const int32_t* counts, int64_t S, int64_t El, int32_t* ids, moe_stream_t stream) {
+  if (!counts || !ids || S < 1 || El < 1) return MOE_ERR_INVALID_ARG;
+  if (S * El > (int64_t(1) << 20)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(counts) & 3u) || (reinterpret_cast<uintptr_t>(ids) & 3u)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_ids_from_counts(counts, int(S), int(El), ids, as_stream(stream)));
 }
 
 moe_status_t moe_check_device_errors(moe_stream_t stream) {

@@ -16,10 +16,17 @@ cudaError_t launch_pack_bitplanes(const uint16_t* w, int64_t E, int64_t N, int64
 cudaError_t launch_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* codes,
                                   uint8_t* block_scales, float* gscale, cudaStream_t st);
 
-// Routing: logits into `logits` (fp32 [T][E]), then top-k and the permutation.
+// Routing: logits into `logits` (fp32 [T][E]), then top-k and the permutation.  The
+// single-launch router elects its last CTA with `counter` (a 32-bit word that must be 0
+// before the launch; the launch leaves it 0).  A workspace holds the counter in its
+// first kRouteCounterBytes and the logits after it.
+constexpr size_t kRouteCounterBytes = 256;
 size_t route_workspace_bytes(int64_t T, int64_t E, int64_t k);
+cudaError_t route_prepare_device();  // per-device kernel attributes; idempotent
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
-                         const moe_routing_t& out, void* ws, cudaStream_t st);
+                         const moe_routing_t& out, float* logits, unsigned* counter, cudaStream_t st);
+cudaError_t launch_route_ws(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                            const moe_routing_t& out, void* ws, cudaStream_t st);
 cudaError_t launch_select_bits(const float* w, int64_t n, const float thr[3], const uint8_t ch[4],
                                uint8_t* bits, cudaStream_t st);
 
@@ -47,6 +54,18 @@ cudaError_t launch_allocate_bits(const double* delta, const double* m, const int
                                  double* lam_out, cudaStream_t st);
 cudaError_t launch_expand_bits(const int32_t* ids, const uint8_t* bits_e, int64_t n, uint8_t* bits,
                                cudaStream_t st);
+
+// Slot cache on the device (moe_cache.cu) and the permutation alone (moe_route.cu).
+cudaError_t launch_permute(const int32_t* ids, int P, int E, const moe_routing_t& out, cudaStream_t st);
+cudaError_t launch_cache_step(void* state, const moe_routing_t& r, const uint8_t* bits, int P, int32_t* slot_ids,
+                              const moe_cache_plan_t& plan, cudaStream_t st);
+cudaError_t launch_cache_fetch(const moe_cache_plan_t& plan, int E, const moe_experts_t& host,
+                               const moe_experts_t& slots, int H, int I, cudaStream_t st);
+
+// Expert parallelism, device side of the exchange (moe_ep.cu).
+cudaError_t launch_gather_rows_by(const uint16_t* src, const int32_t* idx, int n, int div, int H, uint16_t* dst,
+                                  cudaStream_t st);
+cudaError_t launch_ids_from_counts(const int32_t* counts, int S, int El, int32_t* ids, cudaStream_t st);
 
 cudaError_t launch_combine(const uint16_t* y_rows, const moe_routing_t& r, const uint16_t* residual, int T,
                            int H, int k, uint16_t* out, cudaStream_t st);

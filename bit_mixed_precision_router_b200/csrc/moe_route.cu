@@ -255,8 +255,8 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
 // One launch for few tokens: CTA b computes the logits of experts 8b .. 8b+7 for every
 // token (warp = expert; the tokens are staged once in shared memory; the router row's
 // chunks are loaded before any FMA), in the same fixed order as k_router_logits.  The
-// last CTA to finish (ticket counter, reset to 0 by that CTA) reads all logits back,
-// selects every token's top-k and builds the permutation.
+// last CTA to finish (completion counter, reset to 0 by that CTA) reads all logits
+// back, selects every token's top-k and builds the permutation.
 constexpr int kFusedMaxT = 16;
 constexpr int kFusedWarps = 8;
 
@@ -366,8 +366,11 @@ __global__ void k_select_bits(const float* __restrict__ w, int64_t n, float t0, 
 // ---------------------------------------------------------------- launchers
 static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
-// fp32 logits [T][E], then one 32-bit ticket counter (must start at 0; left at 0).
-size_t route_workspace_bytes(int64_t T, int64_t E, int64_t /*k*/) { return align256(size_t(T * E * 4)) + 256; }
+// Workspace: the 32-bit completion counter of k_route_fused in the first 256 bytes (it
+// must start at 0; every fused launch leaves it at 0), then fp32 logits [T][E].  The
+// counter's place does not depend on the shape, so one workspace serves calls of any
+// smaller (T, E) after a larger one.
+size_t route_workspace_bytes(int64_t T, int64_t E, int64_t /*k*/) { return kRouteCounterBytes + align256(size_t(T * E * 4)); }
 
 static bool use_fused(int T, int H, int E, int k) {
   const size_t stage = size_t(T) * H * 2;
@@ -375,27 +378,38 @@ static bool use_fused(int T, int H, int E, int k) {
   return T <= kFusedMaxT && stage <= 64 * 1024 && perm <= 64 * 1024;
 }
 
+// Largest dynamic shared memory the router kernels request: k_route_fused 64 KiB (the
+// tokens, or the permutation's counters), k_permute 33 ints per expert.
+constexpr int kFusedSmemMax = 64 * 1024;
+constexpr int kPermuteSmemMax = 33 * MOE_MAX_EXPERTS * int(sizeof(int));
+
+cudaError_t route_prepare_device() {
+  // once per device: raise both kernels' dynamic shared-memory limit to the largest any
+  // call requests, so no later call (e.g. one inside a stream capture) sets attributes
+  static std::atomic<bool> done[128] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  err = cudaFuncSetAttribute(k_route_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmemMax);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, kPermuteSmemMax);
+  if (err != cudaSuccess) return err;
+  done[dev].store(true, std::memory_order_release);
+  return cudaSuccess;
+}
+
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
-                         const moe_routing_t& out, void* ws, cudaStream_t st) {
-  float* logits = static_cast<float*>(ws);
-  unsigned* ticket = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + align256(size_t(T) * E * 4));
-  cudaError_t err;
+                         const moe_routing_t& out, float* logits, unsigned* counter, cudaStream_t st) {
+  cudaError_t err = route_prepare_device();
+  if (err != cudaSuccess) return err;
   if (use_fused(T, H, E, k)) {
     const size_t stage = size_t(T) * H * 2;
     const size_t perm = size_t(((T * k + 3) & ~3) + kFusedWarps * E + E) * 4;
     const size_t smem = stage > perm ? stage : perm;
-    if (smem > 48 * 1024) {
-      static std::atomic<bool> raised[128] = {};
-      int dev = 0;
-      cudaGetDevice(&dev);
-      if (dev >= 0 && dev < 128 && !raised[dev].load(std::memory_order_relaxed)) {
-        err = cudaFuncSetAttribute(k_route_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-        if (err != cudaSuccess) return err;
-        raised[dev].store(true, std::memory_order_relaxed);
-      }
-    }
     k_route_fused<<<dim3(unsigned((E + kFusedWarps - 1) / kFusedWarps)), 32 * kFusedWarps, smem, st>>>(
-        x, wr, bias, T, H, E, k, logits, ticket, out);
+        x, wr, bias, T, H, E, k, logits, counter, out);
     return cudaGetLastError();
   }
   if (T >= 256) {
@@ -410,12 +424,21 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
   const int P = T * k;
   k_topk<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, out.topk_ids, out.topk_w);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  return launch_permute(out.topk_ids, P, E, out, st);
+}
+
+cudaError_t launch_route_ws(const uint16_t* x, const uint16_t* wr, const float* bias, int T, int H, int E, int k,
+                            const moe_routing_t& out, void* ws, cudaStream_t st) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return launch_route(x, wr, bias, T, H, E, k, out, reinterpret_cast<float*>(base + kRouteCounterBytes),
+                      reinterpret_cast<unsigned*>(base), st);
+}
+
+cudaError_t launch_permute(const int32_t* ids, int P, int E, const moe_routing_t& out, cudaStream_t st) {
+  const cudaError_t err = route_prepare_device();
+  if (err != cudaSuccess) return err;
   const size_t smem = size_t(33 * E) * sizeof(int);
-  if (smem > 48 * 1024) {
-    err = cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (err != cudaSuccess) return err;
-  }
-  k_permute<<<1, 1024, smem, st>>>(out.topk_ids, P, E, out);
+  k_permute<<<1, 1024, smem, st>>>(ids, P, E, out);
   return cudaGetLastError();
 }
 

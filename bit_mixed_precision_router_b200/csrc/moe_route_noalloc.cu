@@ -10,20 +10,23 @@
 // library image instead of a caller-provided workspace.
 //
 // Limits and sharing:
-//   - the array holds kMaxLogits = MOE_NOALLOC_MAX_LOGITS floats (256 KiB) followed
-//     by 256 bytes for the router's completion counter; a call with T * E above
-//     kMaxLogits is rejected with MOE_ERR_UNSUPPORTED_SHAPE;
+//   - the array holds kMaxLogits = MOE_NOALLOC_MAX_LOGITS floats (256 KiB) for the
+//     logits, then 256 bytes whose first word is the one-launch router's completion
+//     counter; a call with T * E above kMaxLogits is rejected with
+//     MOE_ERR_UNSUPPORTED_SHAPE;
+//   - the counter sits at the same place for every shape, after every logit any call
+//     can write, so calls of different shapes in any order find it at zero;
 //   - every GPU that loads the library holds the array until the process exits;
 //   - all calls share it: two calls whose kernels overlap on the same GPU (for
 //     example on two streams) race on it and give undefined routing;
 //   - the logits need no clearing (each call writes every logit it later reads); the
-//     counter, which moe_route_topk expects at zero in the 256 bytes after the
-//     logits, starts at zero because device variables are zero-initialised when the
-//     module loads, and every call leaves it at zero.
+//     counter starts at zero because device variables are zero-initialised when the
+//     module loads, and every call that uses it leaves it at zero.
 // Set-up: the first call on a device looks up the array's device address with
 // cudaGetSymbolAddress (the host-side name is only a stand-in, never a device
-// address) while that device is current, and caches it per device.  Make that
-// first call before capturing a stream into a graph.
+// address) while that device is current, caches it per device, and sets the router
+// kernels' shared-memory attributes for that device.  Make that first call before
+// capturing a stream into a graph; later calls make no set-up call.
 #include <atomic>
 #include <climits>
 
@@ -36,17 +39,19 @@ constexpr int64_t kMaxLogits = MOE_NOALLOC_MAX_LOGITS;
 
 static __device__ __align__(256) float g_route_logits_scratch[kMaxLogits + 64];
 
-// Device address of g_route_logits_scratch on the current device, or nullptr.
+// Device address of g_route_logits_scratch on the current device, or nullptr.  The
+// first call per device also prepares the router kernels for that device.
 float* scratch_on_current_device() {
   static std::atomic<float*> cached[128] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-  float* s = cached[dev].load(std::memory_order_relaxed);
+  float* s = cached[dev].load(std::memory_order_acquire);
   if (!s) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_logits_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_logits_scratch) != cudaSuccess || !p) return nullptr;
+    if (moe::route_prepare_device() != cudaSuccess) return nullptr;
     s = static_cast<float*>(p);
-    cached[dev].store(s, std::memory_order_relaxed);
+    cached[dev].store(s, std::memory_order_release);
   }
   return s;
 }
@@ -73,7 +78,8 @@ extern "C" moe_status_t moe_route_topk_noalloc(const uint16_t* x, const uint16_t
   if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned16(bias))) return MOE_ERR_MISALIGNED;
   float* logits = scratch_on_current_device();
   if (!logits) return MOE_ERR_CUDA;
+  unsigned* counter = reinterpret_cast<unsigned*>(logits + kMaxLogits);  // never reached by a logit write
   const cudaError_t err = moe::launch_route(x, w_router, bias, int(T), int(H), int(E), int(k), *out, logits,
-                                            static_cast<cudaStream_t>(stream));
+                                            counter, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -165,12 +165,15 @@ size_t moe_route_workspace_bytes(int64_t T, int64_t E, int64_t k);
  *   x bf16 [T][H];  w_router bf16 [E][H];  bias fp32 [E] or NULL;  out: see moe_routing_t.
  * Requires H % 256 == 0, 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= min(E, MOE_MAX_TOPK),
  * T >= 0; workspace >= moe_route_workspace_bytes(T, E, k).  Workspace contents: the
- * last 256 bytes of the moe_route_workspace_bytes(T, E, k) region hold a completion
- * counter that must be zero before the first call that uses this workspace (allocate
- * it zero-filled once, e.g. cudaMemset); every call leaves it zero again, so the same
- * workspace serves any number of later calls; the rest is scratch, overwritten.
- * Calls whose kernels overlap on one workspace race on it.  Ids and permutation are
- * deterministic. */
+ * FIRST 256 bytes hold a completion counter (used by the one-launch router of small
+ * batches) that must be zero before the first call that uses this workspace (allocate
+ * it zero-filled once, e.g. cudaMemset); every call leaves it zero again.  The fp32
+ * logits follow it and are scratch, overwritten.  The counter's place does not depend
+ * on (T, E, k), so a workspace sized for (T_max, E_max) serves any number of later
+ * calls of any T <= T_max, E <= E_max, in any order.  Calls whose kernels overlap on
+ * one workspace race on it.  The first call on a device sets the router kernels'
+ * shared-memory attributes for that device (once); make one call before capturing a
+ * stream into a graph.  Ids and permutation are deterministic. */
 moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const float* bias,
                             int64_t T, int64_t H, int64_t E, int64_t k,
                             const moe_routing_t* out, void* workspace, size_t workspace_bytes,
@@ -186,15 +189,17 @@ moe_status_t moe_route_topk(const uint16_t* x, const uint16_t* w_router, const f
  * into a CUDA graph in global mode, where cudaMalloc is not allowed.
  * Same computation, arguments, results and errors as moe_route_topk, except that
  * the fp32 logits scratch and the completion counter are a fixed device array inside
- * the library (256 KiB + 256 bytes per GPU that loads the library, held until exit;
- * the counter is zero when the library loads and every call leaves it zero):
+ * the library (256 KiB + 256 bytes per GPU that loads the library, held until exit):
+ * the logits fill its first T * E floats and the counter is the word right after the
+ * 256 KiB, the same place for every shape (zero when the library loads; every call
+ * leaves it zero), so calls of different shapes may follow one another in any order.
  *   - T * E must be <= MOE_NOALLOC_MAX_LOGITS, else MOE_ERR_UNSUPPORTED_SHAPE;
  *   - the library allocates nothing and frees nothing during the call;
  *   - all calls share the array: calls whose kernels overlap on one GPU (e.g. on two
  *     streams) race on it; serialise them;
  *   - the first call on a device looks up the array's address (cudaGetSymbolAddress
- *     with that device current) and caches it; make that first call before any
- *     stream capture. */
+ *     with that device current), caches it and sets the router kernels' shared-memory
+ *     attributes for that device; make that first call before any stream capture. */
 moe_status_t moe_route_topk_noalloc(const uint16_t* x, const uint16_t* w_router, const float* bias,
                                     int64_t T, int64_t H, int64_t E, int64_t k,
                                     const moe_routing_t* out, moe_stream_t stream);
@@ -283,6 +288,45 @@ moe_status_t moe_cache_plan(void* state, const uint8_t* need, int32_t* served_ex
 /* The slots' contents: expert_of int32 [S] (-1 = free) and resident planes uint8 [S]. */
 moe_status_t moe_cache_slots(const void* state, int32_t* expert_of, uint8_t* planes);
 
+/* ------------------------------------------------------------------------
+ * Expert slot cache on the device (device memory; graph-capturable, no host sync)
+ * ------------------------------------------------------------------------ */
+
+/* One step's plan on the device (device arrays, caller-allocated). */
+typedef struct {
+  int32_t* served_expert; /* [E]  routed experts in ascending id */
+  int32_t* served_slot;   /* [E]  their slots */
+  uint8_t* fetch_lo;      /* [E]  planes [lo, hi) to copy; lo == hi: nothing */
+  uint8_t* fetch_hi;      /* [E] */
+  int32_t* nserved;       /* [1]  number of routed experts */
+  int32_t* overflow;      /* [1]  1 if the step needed more slots than exist (state unchanged) */
+} moe_cache_plan_t;
+
+/* Plans one step on a DEVICE copy of a state written by moe_cache_init (same bytes,
+ * 8-byte aligned device memory), from the routing of the step: need[e] = the largest
+ * bits[p] over e's pairs (bits NULL: 1 for whole experts), and writes every pair's slot
+ * id (slot_ids int32 [T*k]) for moe_permute.  Requires S >= min(E, T*k): one round, in
+ * which the plan equals moe_cache_plan's (no routed expert is evicted); E and S must be
+ * the state's. */
+moe_status_t moe_cache_step(void* state, int64_t E, int64_t S, const moe_routing_t* routing, const uint8_t* bits,
+                            int64_t T, int64_t k, int32_t* slot_ids, const moe_cache_plan_t* plan,
+                            moe_stream_t stream);
+
+/* Copies the planned planes of the served experts from the host store into their slots,
+ * with the expert's scales (and NVFP4 per-expert scale) on a miss.  host_store: the E
+ * experts in the layouts of moe_experts_t, in page-locked host memory the device can read
+ * (cudaHostAlloc, or cudaHostRegister with mapping); slots: the same layouts with S
+ * experts, device memory.  Reads over the host link; returns without waiting. */
+moe_status_t moe_cache_fetch(const moe_cache_plan_t* plan, int64_t E, const moe_experts_t* host_store,
+                             const moe_experts_t* slots, int64_t H, int64_t I, moe_stream_t stream);
+
+/* The permutation of moe_route_topk alone: from ids int32 [T*k] (each < E) writes
+ * out->expert_offsets, sorted_pair, pair_to_row and expert_list (out->topk_ids and
+ * topk_w are not touched).  With ids = moe_cache_step's slot ids and E = S, the routing
+ * of the slot store for moe_grouped_ffn and moe_combine.  T = 0: nothing is written. */
+moe_status_t moe_permute(const int32_t* ids, int64_t T, int64_t k, int64_t E, const moe_routing_t* out,
+                         moe_stream_t stream);
+
 /* Per-pair bit-width from the routing weight [MatMoE: precision per expert from
  * routing scores; PagedMoE: prefix length from current routing weights].
  * bits[p] = choices[0] if w < thresholds[0], choices[1] if w < thresholds[1],
@@ -338,6 +382,24 @@ moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
 moe_status_t moe_combine(const uint16_t* y_rows, const moe_routing_t* routing,
                          const uint16_t* residual, int64_t T, int64_t H, int64_t k,
                          uint16_t* out, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism: the device side of the exchange [ExactMoE: every selected expert
+ * is executed, wherever it is placed].  Rank r owns experts [r E/G, (r+1) E/G); a rank
+ * sends its routed rows in sorted-row order (moe_gather_rows with idx = sorted_pair,
+ * div = k); an owner receives runs in source-rank order, each grouped by local expert,
+ * and labels them with moe_ids_from_counts for moe_permute (k = 1, E = E/G).
+ * ------------------------------------------------------------------------ */
+
+/* dst[i] = src[idx[i] / div] for i < n: rows of H bf16 (H % 8 == 0); idx int32 [n]
+ * (4-byte aligned), every idx[i] / div a valid row of src. */
+moe_status_t moe_gather_rows(const uint16_t* src, const int32_t* idx, int64_t n, int64_t div, int64_t H,
+                             uint16_t* dst, moe_stream_t stream);
+
+/* Local expert of each received row: counts int32 [S][El] (rows from source s for local
+ * expert j); ids int32 [sum of counts] gets j for those rows, ordered by s then j.
+ * One CTA; S * El <= 2^20. */
+moe_status_t moe_ids_from_counts(const int32_t* counts, int64_t S, int64_t El, int32_t* ids, moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Device error reporting

@@ -83,3 +83,38 @@ def check_close(got: np.ndarray, ref: np.ndarray, what: str, atol=ATOL, rel_l2=R
     assert err.max() <= atol, f"{what}: max abs err {err.max():.3e} > {atol}"
     assert rel <= rel_l2, f"{what}: rel L2 err {rel:.3e} > {rel_l2}"
     return float(err.max()), float(rel)
+
+
+def sentinel_routing(moe, T: int, E: int, k: int):
+    """Routing buffers pre-filled with values no call writes (-7, NaN), so that an output
+    a kernel failed to write fails the comparison."""
+    r = moe.Routing.empty(T, E, k)
+    for t in (r.topk_ids, r.expert_offsets, r.sorted_pair, r.pair_to_row, r.expert_list):
+        t.fill_(-7)
+    r.topk_w.fill_(float("nan"))
+    return r
+
+
+def oracle_routing(L: LayerInputs, k: int):
+    """(ids, w, offsets, sorted_pair, pair_to_row) of the oracle for a layer's inputs."""
+    from oracle.routing import permute, router_logits, topk_softmax
+    ids, w = topk_softmax(router_logits(L.x, L.wr, L.bias), k)
+    offsets, sp, p2r = permute(ids, L.E)
+    return ids, w, offsets, sp, p2r
+
+
+def assert_routing_equals_oracle(r, L: LayerInputs, k: int, what: str = ""):
+    """Ids, offsets, sorted_pair, pair_to_row and the active-expert list bit-exact;
+    weights within 1e-6 (CPU exp against the GPU's expf)."""
+    T, E = L.T, L.E
+    ids, w, offsets, sp, p2r = oracle_routing(L, k)
+    P = T * k
+    assert np.array_equal(r.topk_ids.cpu().numpy()[:P].reshape(T, k), ids), f"{what}: topk_ids"
+    got_w = r.topk_w.cpu().numpy()[:P].reshape(T, k)
+    assert np.all(np.isfinite(got_w)) and np.abs(got_w - w).max() <= 1e-6, f"{what}: topk_w"
+    assert np.array_equal(r.expert_offsets.cpu().numpy()[:E + 1], offsets), f"{what}: expert_offsets"
+    assert np.array_equal(r.sorted_pair.cpu().numpy()[:P], sp), f"{what}: sorted_pair"
+    assert np.array_equal(r.pair_to_row.cpu().numpy()[:P], p2r), f"{what}: pair_to_row"
+    el = r.expert_list.cpu().numpy()
+    act = np.nonzero(np.diff(offsets) > 0)[0]
+    assert el[0] == act.size and np.array_equal(el[1:1 + act.size], act), f"{what}: expert_list"

@@ -158,3 +158,34 @@ def test_allocation_validation(lib):
     assert e(4, 8, ids=None) == INVALID
     assert e(4, 8, ids=A + 2) == MISALIGNED
     assert e(0, 8, ids=None) == OK
+
+
+def test_device_cache_validation(lib):
+    plan = moe.CachePlanT(A, A, A, A, A, A)
+    r = RoutingT(A, A, A, A, A, A)
+
+    def step(E, S, T, k, state=A):
+        return lib.moe_cache_step(state, E, S, ctypes.byref(r), None, T, k, A, ctypes.byref(plan), None)
+    assert step(64, 16, 2, 8, state=None) == INVALID
+    assert step(64, 0, 2, 8) == INVALID
+    assert step(64, 65, 2, 8) == INVALID
+    assert step(64, 16, 4, 8) == SHAPE        # 32 pairs may route to 32 experts: more than 16 slots
+    assert step(64, 16, 2, 8, state=A + 4) == MISALIGNED
+    assert step(64, 16, 0, 8) == OK
+    ex = ExpertsT(0, A, A, A, A, None, None)
+
+    def fetch(E, H, I, e1=ex, e2=ex):
+        return lib.moe_cache_fetch(ctypes.byref(plan), E, ctypes.byref(e1), ctypes.byref(e2), H, I, None)
+    assert fetch(64, 2048, 1000) == SHAPE
+    assert fetch(64, 2000, 1024) == SHAPE
+    assert fetch(64, 2048, 1024, e2=ExpertsT(1, A, A, A, A, None, None)) == INVALID   # formats differ
+    nv = ExpertsT(2, A, A, A, A, None, None)
+    assert fetch(64, 2048, 1024, e1=nv, e2=nv) == INVALID                            # NVFP4 needs its scales
+    assert fetch(64, 2048, 1024, e1=ExpertsT(0, A + 8, A, A, A, None, None)) == MISALIGNED
+
+    def perm(T, k, E, ids=A):
+        return lib.moe_permute(ids, T, k, E, ctypes.byref(r), None)
+    assert perm(4, 0, 8) == SHAPE
+    assert perm(4, 2, 8, ids=None) == INVALID
+    assert perm(4, 2, 8, ids=A + 4) == MISALIGNED
+    assert perm(0, 2, 8) == OK

@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import synth
-from layer_inputs import (as_u32, check_close, dev_bf16, host_bits, make_layer, oracle_experts)
+from layer_inputs import (as_u32, assert_routing_equals_oracle, check_close, dev_bf16, host_bits, make_layer,
+                          oracle_experts, sentinel_routing)
 from oracle.ffn import FMT_BITPLANE8, FMT_NVFP4, FMT_W4G128, combine, grouped_ffn
 from oracle.quant import pack_bitplanes, quantize_nvfp4, quantize_w4g128
 from oracle.routing import permute, router_logits, router_logits_f64, select_bits, topk_softmax
@@ -124,7 +125,25 @@ def test_route_workspace_reuse(moe, cuda_device, T, H, E, k):
         offsets, sp, p2r = permute(ids, E)
         assert np.array_equal(out.topk_ids.cpu().numpy().reshape(T, k), ids)
         assert np.array_equal(out.sorted_pair.cpu().numpy(), sp)
-        assert not ws[-256:].any().item()
+        assert not ws[:256].any().item()  # the completion counter, left at zero
+
+
+# (T, E) sequence through one workspace sized for (64, 64): the one-launch router (T <= 16)
+# after larger multi-launch calls, smaller E after larger, and back.
+REUSE_SEQUENCE = [(64, 64), (16, 64), (8, 64), (1, 64), (13, 64), (64, 64), (8, 32), (16, 64), (3, 8), (64, 64)]
+
+
+def test_route_workspace_reuse_across_batches(moe, cuda_device):
+    k = 8
+    ws = moe.moe_route_workspace(64, 64, k, "cuda")
+    for i, (T, E) in enumerate(REUSE_SEQUENCE):
+        kk = min(k, E)
+        L = make_layer(4400 + 31 * i, T, 2048, 128, E, kk, with_experts=False)
+        out = sentinel_routing(moe, T, E, kk)
+        moe.moe_route_topk(dev_bf16(L.x), dev_bf16(L.wr), None, kk, out=out, workspace=ws)
+        moe.moe_check_device_errors()
+        assert_routing_equals_oracle(out, L, kk, f"call {i} (T={T}, E={E})")
+        assert not ws[:256].any().item(), f"call {i}: completion counter not left at zero"
 
 
 def test_route_empty_batch(moe, cuda_device):
