@@ -238,7 +238,9 @@ class DecodeStack:
             self.layers.append((wr, ex))
         del tmp13, tmp2
         B = batch
-        self.routing = moe.Routing.empty(B, E, K_TOP, device)
+        # one routing per layer: after a step every layer's routing is still readable
+        self.routings = [moe.Routing.empty(B, E, K_TOP, device) for _ in range(layers)]
+        self.routing = self.routings[0]
         self.route_ws = moe.moe_route_workspace(B, E, K_TOP, device)
         self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(B, H, I, E, K_TOP, moe.FMT_W4G128), 16),
                                   dtype=torch.uint8, device=device)
@@ -250,16 +252,16 @@ class DecodeStack:
     def layer(self, l, log_active=False):
         moe, wr_ex = self.moe, self.layers[l]
         wr, ex = wr_ex
-        x, nxt = self.xs[l], self.xs[l + 1]
-        moe.moe_route_topk(x, wr, None, K_TOP, out=self.routing, workspace=self.route_ws)
+        x, nxt, r = self.xs[l], self.xs[l + 1], self.routings[l]
+        moe.moe_route_topk(x, wr, None, K_TOP, out=r, workspace=self.route_ws)
         if self.ffn_events is not None:
             self.ffn_events[l][0].record()
-        moe.moe_grouped_ffn(x, self.routing, ex, I, E, K_TOP, y_rows=self.y_rows, workspace=self.ffn_ws)
+        moe.moe_grouped_ffn(x, r, ex, I, E, K_TOP, y_rows=self.y_rows, workspace=self.ffn_ws)
         if self.ffn_events is not None:
             self.ffn_events[l][1].record()
-        moe.moe_combine(self.y_rows, self.routing, self.B, K_TOP, residual=x, out=nxt)
+        moe.moe_combine(self.y_rows, r, self.B, K_TOP, residual=x, out=nxt)
         if log_active:
-            self.n_active[l:l + 1].copy_(self.routing.expert_list[:1])
+            self.n_active[l:l + 1].copy_(r.expert_list[:1])
 
     def step(self, log_active=False):
         for l in range(self.L):

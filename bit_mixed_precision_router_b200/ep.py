@@ -62,6 +62,8 @@ def ep_moe_layer(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor | N
     import torch.distributed as dist
     G = dist.get_world_size(group)
     T, E = x.shape[0], w_router.shape[0]
+    if E % G != 0:
+        raise ValueError(f"{E} experts do not split evenly over {G} ranks")
     El = E // G
     sent = ep_prepare(x, w_router, bias, k)
     recv_counts = torch.empty_like(sent.counts)

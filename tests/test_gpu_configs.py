@@ -83,7 +83,43 @@ class DeviceLayer:
         return out
 
 
-def run_config(moe, fmt, seed, T, H, I, E, k, router="normal", zipf=False, sample=None, bit_rule=False):
+GEMM_ROW_TILE = 192  # routed rows per tile of the tensor-core GEMM path
+
+
+def tile_rows(offsets: np.ndarray, e: int, tile: int = GEMM_ROW_TILE) -> list[int]:
+    """Sorted rows of expert e that cover each of its row tiles: the first and the last
+    row of every tile (the last tile is usually ragged)."""
+    lo, hi = int(offsets[e]), int(offsets[e + 1])
+    rows = []
+    for t0 in range(lo, hi, tile):
+        rows += [t0, min(hi, t0 + tile) - 1]
+    return sorted(set(rows))
+
+
+def pick_experts(offsets: np.ndarray, ids: np.ndarray, tokens, n: int | None) -> list[int]:
+    """Experts whose row tiles are checked: all routed experts (n None), else those of the
+    sampled tokens, the experts with the most and the fewest rows, and evenly spaced
+    ones, n in all (at least)."""
+    counts = np.diff(offsets)
+    routed = [int(e) for e in np.nonzero(counts > 0)[0]]
+    if n is None or n >= len(routed):
+        return routed
+    chosen = {int(e) for t in tokens for e in ids[t]}
+    by_count = sorted(routed, key=lambda e: (counts[e], e))
+    chosen.update(by_count[:2] + by_count[-2:])
+    step = max(1, len(routed) // max(1, n - len(chosen)))
+    for e in routed[::step]:
+        if len(chosen) >= n:
+            break
+        chosen.add(e)
+    return sorted(chosen)
+
+
+def run_config(moe, fmt, seed, T, H, I, E, k, router="normal", zipf=False, sample=None, bit_rule=False,
+               tile_experts: int | None = -1):
+    """tile_experts: -1 checks only the sampled tokens' outputs; None also checks every
+    routed expert's row tiles in y_rows (first and last row of each tile); n checks the
+    row tiles of n experts (pick_experts)."""
     layer = DeviceLayer(moe, fmt, seed, H, I, E)
     x = synth.normal_bf16(seed + synth.SEED_X, T * H, 1.0).reshape(T, H)
     if router == "uniform":
@@ -114,22 +150,58 @@ def run_config(moe, fmt, seed, T, H, I, E, k, router="normal", zipf=False, sampl
         assert np.array_equal(gb[~near], bits[~near])
         bits = np.where(near, gb, bits)  # at a threshold tie both tiers are valid; follow the device
 
-    toks = range(T) if sample is None else sample
-    cache = {}
+    toks = list(range(T)) if sample is None else list(sample)
     got = bf16_to_f64(host_bits(out))
-    worst = (0.0, 0.0)
+    got_y = bf16_to_f64(host_bits(y))
+    xf = bf16_to_f64(x)
+    tile_set = [] if tile_experts == -1 else pick_experts(offsets, ids, toks, tile_experts)
+    need = sorted({int(e) for t in toks for e in ids[t]} | set(tile_set))
+    worst = [0.0, 0.0]
+
+    def expert_check(e, first):
+        deq = layer.host_expert(e, check_device=first)
+        mats = {}
+
+        def ffn(rows_x, b):  # one dequantisation per width
+            if b not in mats:
+                mats[b] = (deq[0](b), deq[1](b))
+            return swiglu_expert(rows_x, *mats[b])
+
+        res = {}
+        rows = tile_rows(offsets, e) if e in tile_set else []
+        pairs = [int(sp[rr]) for rr in rows]
+        for b in sorted({int(bits[p // k, p % k]) if bits is not None else 8 for p in pairs}):
+            sel = [(rr, p) for rr, p in zip(rows, pairs)
+                   if (int(bits[p // k, p % k]) if bits is not None else 8) == b]
+            yr = ffn(xf[[p // k for _, p in sel]], b)
+            for (rr, _), yv in zip(sel, yr):
+                res[rr] = check_close(got_y[rr], yv, f"y_rows row {rr} (expert {e})")
+        # this expert's contribution to the sampled tokens' outputs
+        contrib = {}
+        for t in toks:
+            for j in range(k):
+                if int(ids[t, j]) == e:
+                    b = int(bits[t, j]) if bits is not None else 8
+                    contrib[(t, j)] = ffn(xf[t:t + 1], b)[0]
+        return res, contrib
+
+    import concurrent.futures as cf
+    import os
+    contribs = {}
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as pool:
+        for i0 in range(0, len(need), 16):  # bounded memory: 16 dequantised experts at a time
+            for res, c in pool.map(lambda a: expert_check(*a), [(e, i < 2) for i, e in enumerate(need[i0:i0 + 16],
+                                                                                                  start=i0)]):
+                for m, rel in res.values():
+                    worst = [max(worst[0], m), max(worst[1], rel)]
+                contribs.update(c)
     for t in toks:
         ref = np.zeros(H)
         for j in range(k):
-            e = int(ids[t, j])
-            if e not in cache:
-                cache[e] = layer.host_expert(e, check_device=len(cache) < 2)
-            b = int(bits[t, j]) if bits is not None else 8
-            w13d, w2d = cache[e][0](b), cache[e][1](b)
-            ref += float(w[t, j]) * swiglu_expert(bf16_to_f64(x[t:t + 1]), w13d, w2d)[0]
+            ref += float(w[t, j]) * contribs[(t, j)]
         m, rel = check_close(got[t], ref, f"token {t}")
-        worst = max(worst, (m, rel))
-    return worst
+        worst = [max(worst[0], m), max(worst[1], rel)]
+    return tuple(worst)
 
 
 def test_config_olmoe_layer_16_tokens_w4(moe, cuda_device):
@@ -144,12 +216,17 @@ def test_config_bitplane_64_tokens(moe, cuda_device):
 
 
 def test_config_qwen_prefill_zipf(moe, cuda_device):
-    # H2048 I768 E128 top-8, 2048 tokens with Zipf-skewed routing; all ids, 6 tokens' outputs
-    run_config(moe, FMT_W4G128, 0x5EED0003, 2048, 2048, 768, 128, 8, zipf=True, sample=[0, 1, 777, 1500, 2046, 2047])
+    # H2048 I768 E128 top-8, 2048 tokens with Zipf-skewed routing: all ids; every routed
+    # expert's row tiles (first and last row of each, incl. the ragged last tile) in y_rows;
+    # 6 tokens' combined outputs
+    run_config(moe, FMT_W4G128, 0x5EED0003, 2048, 2048, 768, 128, 8, zipf=True, sample=[0, 1, 777, 1500, 2046, 2047],
+               tile_experts=None)
 
 
 @pytest.mark.parametrize("fmt", [FMT_W4G128, FMT_NVFP4])
-@pytest.mark.parametrize("T,sample", [(1, None), (64, [0, 63]), (4096, [4095])])
-def test_config_deepseek_v3_like(moe, cuda_device, fmt, T, sample):
-    # H7168 I2048 E256 top-8, uniform-random router weights
-    run_config(moe, fmt, 0x5EED0005, T, 7168, 2048, 256, 8, router="uniform", sample=sample)
+@pytest.mark.parametrize("T,sample,tiles", [(1, None, -1), (64, [0, 63], None), (4096, [4095], 24)])
+def test_config_deepseek_v3_like(moe, cuda_device, fmt, T, sample, tiles):
+    # H7168 I2048 E256 top-8, uniform-random router weights.  T=64: every routed expert's
+    # rows; T=4096: the row tiles of 24 experts (the sampled token's, the largest and
+    # smallest, evenly spaced ones)
+    run_config(moe, fmt, 0x5EED0005, T, 7168, 2048, 256, 8, router="uniform", sample=sample, tile_experts=tiles)
