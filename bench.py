@@ -47,19 +47,26 @@ W4_EXPERT_BYTES = (2 * I * H + H * I) // 2 + (2 * I * (H // 128) + H * (I // 128
 W13_EXPERT_BYTES = 2 * I * H // 2 + 2 * I * (H // 128) * 2
 W2_EXPERT_BYTES = H * I // 2 + H * (I // 128) * 2
 
-# Prefill-sized single layers (W4A16 g128 experts): shapes, routing and seeds.
-PREFILL = {
+# Single-layer workloads (one MoE FFN layer per step on fresh tokens): shapes, routing,
+# weight format and seeds.  Decode-sized batches run the weight-streaming GEMV path
+# (HBM-bound), prefill-sized ones (T*k >= 32*E, W4 or NVFP4) the tensor-core GEMM path.
+_DSV3 = dict(H=7168, I=2048, E=256, k=8, router="uniform", zipf=False, seed=0x5EED0005)
+_DSV3_DESC = ("one MoE FFN layer, H7168 I2048 E256 top-8, %s experts, U(-0.02, 0.02) bf16 router, "
+              "%d fresh tokens per step")
+_W4, _FP4 = "W4A16 g128", "NVFP4 (E2M1, E4M3 per 16, fp32 per tensor)"
+LAYER_WORKLOADS = {
+    "layer-h2048-e64-t16": dict(T=16, H=2048, I=1024, E=64, k=8, router="normal", zipf=False, seed=0x5EED0001,
+                                desc="one MoE FFN layer, H2048 I1024 E64 top-8, W4A16 g128 experts, bf16 router, "
+                                     "16 fresh tokens per step"),
     "prefill-h2048-e128": dict(T=2048, H=2048, I=768, E=128, k=8, router="normal", zipf=True, seed=0x5EED0003,
                                desc="one MoE FFN layer, H2048 I768 E128 top-8, W4A16 g128 experts, bf16 router "
                                     "with a Zipf(1.1) rank bias, 2048 fresh tokens per step"),
-    "prefill-h7168-e256": dict(T=4096, H=7168, I=2048, E=256, k=8, router="uniform", zipf=False, seed=0x5EED0005,
-                               desc="one MoE FFN layer, H7168 I2048 E256 top-8, W4A16 g128 experts, "
-                                    "U(-0.02, 0.02) bf16 router, 4096 fresh tokens per step"),
-    "prefill-h7168-e256-nvfp4": dict(T=4096, H=7168, I=2048, E=256, k=8, router="uniform", zipf=False,
-                                     seed=0x5EED0005, fmt="nvfp4",
-                                     desc="one MoE FFN layer, H7168 I2048 E256 top-8, NVFP4 experts (E2M1, E4M3 "
-                                          "per 16, fp32 per tensor), U(-0.02, 0.02) bf16 router, 4096 fresh "
-                                          "tokens per step"),
+    "layer-h7168-e256-t1": dict(T=1, desc=_DSV3_DESC % (_W4, 1), **_DSV3),
+    "layer-h7168-e256-t64": dict(T=64, desc=_DSV3_DESC % (_W4, 64), **_DSV3),
+    "prefill-h7168-e256": dict(T=4096, desc=_DSV3_DESC % (_W4, 4096), **_DSV3),
+    "layer-h7168-e256-t1-nvfp4": dict(T=1, fmt="nvfp4", desc=_DSV3_DESC % (_FP4, 1), **_DSV3),
+    "layer-h7168-e256-t64-nvfp4": dict(T=64, fmt="nvfp4", desc=_DSV3_DESC % (_FP4, 64), **_DSV3),
+    "prefill-h7168-e256-nvfp4": dict(T=4096, fmt="nvfp4", desc=_DSV3_DESC % (_FP4, 4096), **_DSV3),
     "bitplane-h2048-e64": dict(T=64, H=2048, I=1024, E=64, k=8, router="normal", zipf=False, seed=0x5EED0004,
                                fmt="bitplane", bits="rule",
                                desc="one MoE FFN layer, H2048 I1024 E64 top-8, 8-bitplane experts, each "
@@ -73,6 +80,13 @@ PREFILL = {
                                             "routing-weighted reads over {2,3,4,8}, profiled on 2048 tokens), "
                                             "bf16 router, 64 fresh tokens per step"),
 }
+PREFILL = LAYER_WORKLOADS
+
+# The records the default run adds to its line (`workloads`), one per benchmark
+# configuration besides the headline decode stack at batch 8.
+EXTRA_WORKLOADS = ["decode-b1", "layer-h2048-e64-t16", "prefill-h2048-e128", "bitplane-h2048-e64",
+                   "bitplane-h2048-e64-duorate", "layer-h7168-e256-t1", "layer-h7168-e256-t64", "prefill-h7168-e256",
+                   "layer-h7168-e256-t1-nvfp4", "layer-h7168-e256-t64-nvfp4", "prefill-h7168-e256-nvfp4"]
 # bitplane experts: bytes of one plane of one expert's w13 + w2, and of their bf16 scales
 BP_PLANE_BYTES = (2 * I * H + H * I) // 8
 BP_SCALE_BYTES = (2 * I * (H // 128) + H * (I // 128)) * 2
@@ -81,7 +95,10 @@ BP_SCALE_BYTES = (2 * I * (H // 128) + H * (I // 128)) * 2
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--workload", choices=["decode"] + sorted(PREFILL), default="decode")
+    ap.add_argument("--workload", choices=["decode"] + sorted(LAYER_WORKLOADS), default="decode")
+    ap.add_argument("--workloads", choices=["all", "none"], default="all",
+                    help="with the default decode workload at N=1: also time every other benchmark "
+                         "configuration and add one record each to the line (`workloads`)")
     ap.add_argument("--steps", type=int, default=None, help="timed steps (default 512 decode, 20 prefill)")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--batch", type=int, default=8)
@@ -95,8 +112,14 @@ def parse_args(argv=None):
                     help="layers in the stack (16 is the benchmark workload; fewer only for profiling)")
     args = ap.parse_args(argv)
     if args.steps is None:
-        args.steps = 512 if args.workload == "decode" or args.workload.startswith("bitplane") else 20
+        args.steps = default_steps(args.workload)
     return args
+
+
+def default_steps(workload: str) -> int:
+    if workload == "decode":
+        return 512
+    return 20 if LAYER_WORKLOADS[workload]["T"] >= 2048 else 512 if workload.startswith("bitplane") else 200
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -366,15 +389,44 @@ def run_gpu(args, rank, world, local):
     init_dist(world, "nccl")
     import bit_mixed_precision_router_b200 as moe
     moe.load()
-    import synth
+    W = max(args.warmup, 3)
+    rec = bench_stack(moe, torch, device, args.batch, args.steps, W, rank, world, local, args.layers,
+                      e2e=not args.no_e2e, cache_slots=args.cache_slots)
+    extra = []
+    if world == 1 and args.workloads == "all" and not args.cache_slots and args.layers == LAYERS:
+        for name in EXTRA_WORKLOADS:
+            try:
+                if name == "decode-b1":
+                    r = bench_stack(moe, torch, device, 1, 512, W, rank, world, local, LAYERS, e2e=not args.no_e2e)
+                else:
+                    r = bench_layer(moe, torch, device, LAYER_WORKLOADS[name], default_steps(name), W, rank, world,
+                                    local, e2e=not args.no_e2e)
+            except Exception as exc:  # a failed record is reported, the others still run
+                r = {"error": f"{type(exc).__name__}: {exc}"}
+                torch.cuda.empty_cache()
+            r["name"] = name
+            extra.append(r)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    line = line_from_record(rec, world)
+    if extra:
+        line["workloads"] = extra
+    return line
 
-    B, K, W = args.batch, args.steps, max(args.warmup, 3)
+
+def bench_stack(moe, torch, device, B, K, W, rank, world, local, L, e2e=True, cache_slots=0):
+    """Times the decode stack: K replays of one CUDA graph holding all L layers, each step on
+    a fresh seeded batch of B tokens resident in HBM; then the same through pinned host
+    buffers (e2e); then the dominant op's roofline."""
+    import synth
     seed = rank_seed(SEED_BASE, rank)
-    L = args.layers
-    if args.cache_slots:
-        if not (1 <= args.cache_slots <= E and args.cache_slots >= min(E, B * K_TOP)):
+    if cache_slots:
+        if not (1 <= cache_slots <= E and cache_slots >= min(E, B * K_TOP)):
             raise SystemExit("--cache-slots must be in [min(E, batch * top-k), E]")
-        stack = CachedDecodeStack(moe, torch, device, B, seed, L, args.cache_slots)
+        stack = CachedDecodeStack(moe, torch, device, B, seed, L, cache_slots)
     else:
         stack = DecodeStack(moe, torch, device, B, seed, L)
     # a fresh seeded N(0,1) batch for every step (warm-up and timed), resident in HBM
@@ -425,8 +477,8 @@ def run_gpu(args, rank, world, local):
     value = tokens / (ms / 1e3)
 
     # ---- end-to-end through the public API with host buffers (pinned), copies timed
-    e2e = None
-    if not args.no_e2e:
+    e2e_rec = None
+    if e2e:
         host_in = inputs.cpu().pin_memory()
         host_out = torch.empty((K, B, H), dtype=torch.bfloat16).pin_memory()
         barrier(world)
@@ -441,38 +493,34 @@ def run_gpu(args, rank, world, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
-        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": B * H * 2,
-               "d2h_bytes_per_step": B * H * 2}
+        e2e_rec = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": B * H * 2,
+                   "d2h_bytes_per_step": B * H * 2}
 
-    if args.cache_slots:
+    if cache_slots:
         roofline, act = cached_roofline(torch, device, stack, cap, inputs, W, K)
     else:
         roofline, act = resident_roofline(torch, stack, cap, inputs, W, K, B)
-    result = None
-    if rank == 0:
-        cfg_extra = {} if not args.cache_slots else {
-            "cache": "experts of each layer in pinned host memory, %d device slots per layer, planned on the "
-                     "device each step, missing experts read over the host link" % args.cache_slots}
-        result = {
-            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, "
-                                                          "N(0,0.02) bf16 weights quantised to W4A16 g128)",
-            "config": dict({"workload": "decode stack: %d chained OLMoE-like MoE FFN layers (H2048 I1024 E64 "
-                                        "top-8, W4A16 g128 experts, bf16 router), residual add, batch %d "
-                                        "tokens/step" % (L, B),
-                            "layers": L, "batch": B, "hidden": H, "intermediate": I, "experts": E, "top_k": K_TOP,
-                            "parallelism": f"dp{world} (independent replicas)",
-                            "l2": "no flush: each step streams ~%.1f GB of distinct expert weights, > 126 MB L2"
-                                  % (statistics.mean(act) * W4_EXPERT_BYTES * L / 1e9)}, **cfg_extra),
-            "gpu_launches": stack.kernels_per_step * K,
-            "clocks": clk, "roofline": roofline, "e2e": e2e,
-        }
-    if world > 1:
-        import torch.distributed as dist
-        del graph
-        dist.destroy_process_group()
-    return result
+    cfg_extra = {} if not cache_slots else {
+        "cache": "experts of each layer in pinned host memory, %d device slots per layer, planned on the "
+                 "device each step, missing experts read over the host link" % cache_slots}
+    rec = {
+        "value": round(value, 1), "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
+        "dtype": "bf16", "data": "synthetic (seeded Irwin-Hall N(0,1) activations, N(0,0.02) bf16 weights "
+                                 "quantised to W4A16 g128)",
+        "config": dict({"workload": "decode stack: %d chained OLMoE-like MoE FFN layers (H2048 I1024 E64 "
+                                    "top-8, W4A16 g128 experts, bf16 router), residual add, batch %d "
+                                    "tokens/step" % (L, B),
+                        "layers": L, "batch": B, "hidden": H, "intermediate": I, "experts": E, "top_k": K_TOP,
+                        "parallelism": f"dp{world} (independent replicas)",
+                        "l2": "no flush: each step streams ~%.1f GB of distinct expert weights, > 126 MB L2"
+                              % (statistics.mean(act) * W4_EXPERT_BYTES * L / 1e9)}, **cfg_extra),
+        "gpu_launches": stack.kernels_per_step * K,
+        "clocks": clk, "roofline": roofline, "e2e": e2e_rec,
+    }
+    del graph, stack, inputs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def cached_roofline(torch, device, stack, cap, inputs, W, K):
@@ -540,10 +588,35 @@ def resident_roofline(torch, stack, cap, inputs, W, K, B):
     return roofline, act
 
 
-# ---------------------------------------------------------------- prefill workloads
+# ---------------------------------------------------------------- single-layer workloads
+L2_BYTES = 126 * 1000 ** 2
+
+
+def expert_bytes(cfg) -> int:
+    """Packed weights + scales of one expert (w13 and w2) in the workload's format."""
+    n = 3 * cfg["H"] * cfg["I"]  # weights per expert
+    fmt = cfg.get("fmt")
+    if fmt == "nvfp4":
+        return n // 2 + n // 16 + 8
+    if fmt == "bitplane":
+        return n + n // 128 * 2
+    return n // 2 + n // 128 * 2
+
+
+def gemm_path(cfg) -> bool:
+    """moe_grouped_ffn's own choice: the tensor-core GEMM for W4 / NVFP4 batches with
+    T*k >= 32*E, else the weight-streaming GEMV."""
+    return cfg.get("fmt") != "bitplane" and cfg["T"] * cfg["k"] >= 32 * cfg["E"]
+
+
+def fused_router(T: int, Hh: int) -> bool:
+    return T <= 16 and T * Hh * 2 <= 64 * 1024
+
+
 class PrefillLayer:
-    """One W4A16 MoE FFN layer made on the device (seeded generator, quantised in
-    chunks of experts) with every buffer a prefill step needs."""
+    """One MoE FFN layer made on the device (seeded generator, quantised in chunks of
+    experts) with every buffer a step needs.  Steps rotate over device copies of the
+    weights where one copy would sit in the 126 MB L2 between steps."""
 
     def __init__(self, moe, torch, device, cfg, chunk=16):
         import synth
@@ -592,15 +665,19 @@ class PrefillLayer:
         self.out = torch.empty((T, Hh), **bf)
         self.ffn_events = None
         self.bits_e = self.bits = None
-        self.copies = [self.experts]
+        self.n_active = torch.zeros((1,), **i32)
         if self.fmt == moe.FMT_BITPLANE8:
             self.bits = torch.empty((T * k,), **u8)
-            # a step reads only ~b_e planes of each expert (about 160 MB, near the 126 MB L2):
-            # steps rotate over 4 device copies of the same weights so no step finds the
-            # previous step's planes in L2
-            for _ in range(3):
-                self.copies.append(moe.Experts(self.fmt, w13[0].clone(), w13[1].clone(), w2[0].clone(),
-                                               w2[1].clone(), None, None))
+        # copies of the weights to rotate over: a step of the bitplane layer reads ~160 MB of
+        # planes, the H2048 W4 layer ~180 MB of its 207 MB, near the 126 MB L2; 4 * L2 bytes
+        # in rotation make sure no step finds the previous steps' weights in L2
+        total = Ee * expert_bytes(cfg)
+        n_copies = 4 if self.fmt == moe.FMT_BITPLANE8 else max(1, min(4, -(-4 * L2_BYTES // total)))
+        self.copies = [self.experts]
+        g = lambda t: None if t is None else t.clone()
+        for _ in range(n_copies - 1):
+            self.copies.append(moe.Experts(self.fmt, w13[0].clone(), w13[1].clone(), w2[0].clone(), w2[1].clone(),
+                                           g(w13[2]), g(w2[2])))
 
     def allocate_widths(self, torch, device, seed):
         """Per-expert widths for the bitplane experts under the read budget: the distortion
@@ -640,7 +717,7 @@ class PrefillLayer:
                 "resident_rate_mean_width": round(float(be.double().mean()), 4), "lambda": lam.item(),
                 "kernel_us": {key: round(statistics.median(v), 1) for key, v in times.items()}}
 
-    def step(self, copy: int = 0):
+    def step(self, copy: int = 0, log_active: bool = False):
         moe, c = self.moe, self.cfg
         moe.moe_route_topk(self.x, self.wr, self.bias, c["k"], out=self.routing, workspace=self.route_ws)
         if self.bits is not None:
@@ -655,26 +732,51 @@ class PrefillLayer:
         if self.ffn_events is not None:
             self.ffn_events[1].record()
         moe.moe_combine(self.y_rows, self.routing, c["T"], c["k"], residual=self.x, out=self.out)
+        if log_active:
+            self.n_active.copy_(self.routing.expert_list[:1])
 
     @property
     def kernels_per_step(self):
-        # router logits, top-k, permutation (the one-launch router only takes <= 16 tokens of
-        # <= 64 KiB), then the row gather + gate/up + down of the tensor-core path, or
-        # (bitplanes) the width expansion + gate/up + down GEMV, then the combine
-        return 3 + 3 + 1
+        c = self.cfg
+        route = 1 if fused_router(c["T"], c["H"]) else 3  # logits + top-k + permutation otherwise
+        widths = 1 if self.bits is not None else 0        # select_bits / expand_bits
+        ffn = 3 if gemm_path(c) else 2                    # (row gather +) gate/up + down
+        return route + widths + ffn + 1                   # + combine
 
 
 def run_prefill(args, rank, world, local):
+    """A single-layer workload as the line's main measurement (`--workload`)."""
     import torch
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
     import bit_mixed_precision_router_b200 as moe
     moe.load()
+    rec = bench_layer(moe, torch, device, LAYER_WORKLOADS[args.workload], args.steps, max(args.warmup, 3), rank,
+                      world, local, e2e=not args.no_e2e)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return line_from_record(rec, world)
+
+
+def line_from_record(rec, world):
+    """The contract's JSON line from a workload record."""
+    out = {"metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world, "steps": rec["steps"],
+           "warmup": rec["warmup"], "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None}
+    out.update({k: v for k, v in rec.items() if k not in out and k != "name"})
+    return out
+
+
+def bench_layer(moe, torch, device, cfg, K, W, rank, world, local, e2e=True):
+    """Times one single-layer workload: K graph replays (W warm-up), each a step on fresh
+    tokens resident in HBM; then the same through pinned host buffers (e2e); then the
+    dominant op's roofline from CUDA events around moe_grouped_ffn inside a graph."""
     import synth
-    cfg = PREFILL[args.workload]
     T, Hh, Ii, Ee, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
-    K, W = args.steps, max(args.warmup, 3)
     layer = PrefillLayer(moe, torch, device, cfg)
     allocation = layer.allocate_widths(torch, device, rank_seed(cfg["seed"], rank)) \
         if cfg.get("bits") == "allocated" else None
@@ -716,8 +818,8 @@ def run_prefill(args, rank, world, local):
     tokens = T * K * world
     value = tokens / (ms / 1e3)
 
-    e2e = None
-    if not args.no_e2e:
+    e2e_rec = None
+    if e2e:
         host_in = inputs[W:W + K].cpu().pin_memory()
         host_out = torch.empty((K, T, Hh), dtype=torch.bfloat16).pin_memory()
         barrier(world)
@@ -732,22 +834,25 @@ def run_prefill(args, rank, world, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
-        e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * Hh * 2,
-               "d2h_bytes_per_step": T * Hh * 2}
+        e2e_rec = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": T * Hh * 2,
+                   "d2h_bytes_per_step": T * Hh * 2}
 
-    # roofline of the dominant op: the grouped GEMM (row gather + gate/up + down launches
-    # of moe_grouped_ffn), CUDA events recorded on its stream inside a graph
+    # roofline of the dominant op: one moe_grouped_ffn call (the row gather + two tcgen05
+    # GEMMs, or the two GEMV launches), CUDA events recorded on its stream inside a graph
     layer.ffn_events = (torch.cuda.Event(enable_timing=True, external=True),
                         torch.cuda.Event(enable_timing=True, external=True))
     g2s = [torch.cuda.CUDAGraph() for _ in range(nc)]
     with torch.cuda.stream(cap):
         for c_, g2 in enumerate(g2s):
             with torch.cuda.graph(g2, stream=cap):
-                layer.step(c_)
+                layer.step(c_, log_active=True)
     torch.cuda.current_stream().wait_stream(cap)
     ffn_ms, ffn_bytes = [], []
     bitplane = layer.bits is not None
-    for s in range(W, W + min(K, 10)):
+    gemm = gemm_path(cfg)
+    act_bytes = T * Hh * 2 + T * k * Ii * 2 * 2 + T * k * Hh * 2  # x, h (written and read), y_rows
+    n_meas = min(K, 10 if gemm else 64)
+    for s in range(W, W + n_meas):
         layer.x.copy_(inputs[s])
         g2s[s % nc].replay()
         torch.cuda.synchronize()
@@ -763,53 +868,57 @@ def run_prefill(args, rank, world, local):
                 if offs[e + 1] > offs[e]:
                     bmax = max(bits[sp[r]] for r in range(offs[e], offs[e + 1]))
                     nbytes += bmax * BP_PLANE_BYTES + BP_SCALE_BYTES
-            ffn_bytes.append(nbytes)
+            ffn_bytes.append(nbytes + act_bytes)
+        else:
+            ffn_bytes.append(int(layer.n_active.item()) * expert_bytes(cfg) + act_bytes)
     layer.ffn_events = None
     hbm, bf16_peak, peak_kind = measured_peaks()
     avg_s = statistics.mean(ffn_ms) / 1e3
-    if bitplane:
-        achieved = sum(ffn_bytes) / (sum(ffn_ms) / 1e3) / 1e9
-        tr = committed_traffic("traffic_bitplane.json") if allocation is not None else None
-        # DRAM bytes of one captured call (all 64 experts at 3 planes, as the allocated workload reads)
-        traffic = tr["dram_bytes_per_call"] if tr else None
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved / hbm, 4), "peak_kind": peak_kind + " HBM copy", "traffic": traffic,
-                    "kernel": "k_ffn_gemv<bitplane> gate/up + down (one moe_grouped_ffn call)",
-                    "algorithmic_bytes_per_call": round(statistics.mean(ffn_bytes)),
-                    "avg_call_us": round(avg_s * 1e6, 1)}
-    else:
+    if gemm:
         flops = 2.0 * T * k * 3 * Hh * Ii
         achieved = flops / avg_s / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
-                    "frac": round(achieved / bf16_peak, 4), "peak_kind": peak_kind + " bf16 burst",
+                    "frac": round(achieved / bf16_peak, 4),
+                    "peak_kind": peak_kind + " bf16 burst" + (" (the fp16 MMAs of this path have the same dense "
+                                                              "peak)" if cfg.get("fmt") == "nvfp4" else ""),
                     "traffic": None,
                     "kernel": "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
                     "algorithmic_flops_per_call": flops, "avg_call_us": round(avg_s * 1e6, 1)}
-    result = None
-    if rank == 0:
-        result = {
-            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp16" if cfg.get("fmt") == "nvfp4" else "bf16",
-            "data": "synthetic (seeded Irwin-Hall N(0,1) activations, N(0,0.02) bf16 weights quantised to "
-                    + {"nvfp4": "NVFP4", "bitplane": "8 bitplanes"}.get(cfg.get("fmt"), "W4A16 g128") + ")",
-            "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,
-                       "top_k": k, "parallelism": f"dp{world} (independent replicas)",
-                       "l2": ("no flush: each step reads more than %.1f GB of expert weights, > 126 MB L2"
-                              % (Ee * 3 * Hh * Ii / 2 / 1e9)) if not bitplane else
-                             ("no flush: each step reads about %.0f MB of expert planes and scales, and "
-                              "steps rotate over 4 device copies of the weights (> 126 MB L2 between "
-                              "reuses)" % (statistics.mean(ffn_bytes) / 1e6))},
-            "gpu_launches": layer.kernels_per_step * K,
-            "clocks": clk, "roofline": roofline, "e2e": e2e,
-        }
+    else:
+        achieved = sum(ffn_bytes) / (sum(ffn_ms) / 1e3) / 1e9
+        traffic = None
         if allocation is not None:
-            result["config"]["allocation"] = allocation
-    if world > 1:
-        import torch.distributed as dist
-        del graphs, g2s
-        dist.destroy_process_group()
-    return result
+            tr = committed_traffic("traffic_bitplane.json")
+            traffic = tr["dram_bytes_per_call"] if tr else None  # all 64 experts at 3 planes, as allocated
+        fmt_name = {"nvfp4": "NVFP4", "bitplane": "bitplane"}.get(cfg.get("fmt"), "W4")
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4), "peak_kind": peak_kind + " HBM copy", "traffic": traffic,
+                    "kernel": f"k_ffn_gemv<{fmt_name}> gate/up + down (one moe_grouped_ffn call)",
+                    "algorithmic_bytes_per_call": round(statistics.mean(ffn_bytes)),
+                    "avg_call_us": round(avg_s * 1e6, 1)}
+    fmt = cfg.get("fmt")
+    if bitplane:
+        l2 = ("no flush: each step reads about %.0f MB of expert planes and scales, and steps rotate over %d "
+              "device copies of the weights (> 4 x 126 MB L2 between reuses)" % (statistics.mean(ffn_bytes) / 1e6, nc))
+    elif nc > 1:
+        l2 = ("no flush: steps rotate over %d device copies of the %.0f MB of expert weights (> 4 x 126 MB L2 "
+              "between reuses)" % (nc, Ee * expert_bytes(cfg) / 1e6))
+    else:
+        l2 = "no flush: the %.1f GB of expert weights exceed 4 x the 126 MB L2" % (Ee * expert_bytes(cfg) / 1e9)
+    rec = {"value": round(value, 1), "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
+           "dtype": "fp16" if fmt == "nvfp4" and gemm else "bf16",
+           "data": "synthetic (seeded Irwin-Hall N(0,1) activations, N(0,0.02) bf16 weights quantised to "
+                   + {"nvfp4": "NVFP4", "bitplane": "8 bitplanes"}.get(fmt, "W4A16 g128") + ")",
+           "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,
+                      "top_k": k, "path": "tcgen05 grouped GEMM" if gemm else "grouped GEMV",
+                      "parallelism": f"dp{world} (independent replicas)", "l2": l2},
+           "gpu_launches": layer.kernels_per_step * K, "clocks": clk, "roofline": roofline, "e2e": e2e_rec}
+    if allocation is not None:
+        rec["config"]["allocation"] = allocation
+    del graphs, g2s, layer, inputs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def oracle_prefill_sample(cfg, tokens: int, seed: int):
@@ -921,25 +1030,69 @@ def prefill_sample_tokens(cfg) -> int:
         return 1
     if cfg.get("fmt") == "bitplane":
         return 16
-    return 2 if cfg["H"] > 4096 else 32
+    return 2 if cfg["H"] > 4096 else min(cfg["T"], 32)
 
 
-def cpu_baseline_prefill(cfg, seed: int):
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _one_thread(fn):
+    """fn() with every BLAS / OpenMP pool limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        return fn()
+
+
+def cpu_baseline_prefill(cfg, seed: int, one_thread: bool = False):
     n = prefill_sample_tokens(cfg)
     v, secs, thr = oracle_prefill_sample(cfg, n, seed)
-    return {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
-            "sample": f"{n} tokens through the layer ({secs:.1f} s of CPU work: routing, dequantisation of "
-                      f"their experts" + (" at 3 planes each" if cfg.get("bits") == "allocated" else
-                                          " at the thresholds' widths" if cfg.get("fmt") == "bitplane" else "")
-                      + ", SwiGLU, combine); weights generated and quantised untimed"}
+    out = {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "host_threads": os.cpu_count(), "kind": "oracle",
+           "sample": f"{n} tokens through the layer ({secs:.1f} s of CPU work: routing, dequantisation of "
+                     f"their experts" + (" at 3 planes each" if cfg.get("bits") == "allocated" else
+                                         " at the thresholds' widths" if cfg.get("fmt") == "bitplane" else "")
+                     + ", SwiGLU, combine); weights generated and quantised untimed"}
+    if one_thread:
+        v1, secs1, _ = _one_thread(lambda: oracle_prefill_sample(cfg, n, seed))
+        out["value_1thread"] = round(v1, 3)
+    return out
 
 
-def cpu_baseline(batch: int, seed: int):
+def cpu_baseline(batch: int, seed: int, one_thread: bool = False):
     layers_timed = 2
     v, secs, thr = oracle_sample(batch, layers_timed, seed)
-    return {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "kind": "oracle",
-            "sample": f"{layers_timed} of the 16 layers of one decode step at batch {batch} "
-                      f"({secs:.1f} s of CPU work), scaled to the full step"}
+    out = {"value": round(v, 3), "unit": "tokens/s", "cores": thr, "host_threads": os.cpu_count(), "kind": "oracle",
+           "sample": f"{layers_timed} of the 16 layers of one decode step at batch {batch} "
+                     f"({secs:.1f} s of CPU work), scaled to the full step"}
+    if one_thread:
+        v1, secs1, _ = _one_thread(lambda: oracle_sample(batch, layers_timed, seed))
+        out["value_1thread"] = round(v1, 3)
+        out["sample"] += f"; the same sample on one thread took {secs1:.1f} s"
+    return out
+
+
+def cpu_baselines_for(records) -> None:
+    """Adds the oracle's CPU baseline to each workload record.  The single-layer workloads
+    of one layer shape and format share one oracle measurement (tokens/s per token of that
+    layer, the same at every batch size: the oracle evaluates token by token)."""
+    shared = {}
+    for r in records:
+        if "error" in r:
+            continue
+        name = r["name"]
+        if name == "decode-b1":
+            r["cpu_baseline"] = cpu_baseline(1, SEED_BASE)
+            continue
+        cfg = LAYER_WORKLOADS[name]
+        key = (cfg["H"], cfg["I"], cfg["E"], cfg.get("fmt"), cfg.get("bits"), cfg["zipf"], cfg["router"])
+        if key not in shared:
+            shared[key] = cpu_baseline_prefill(cfg, cfg["seed"])
+            shared[key]["measured_on"] = name
+        r["cpu_baseline"] = dict(shared[key])
 
 
 def run_reference(args, rank, world):
@@ -991,14 +1144,16 @@ def main(argv=None):
     if args.workload != "decode":
         res = run_prefill(args, rank, world, local)
         if rank == 0 and res is not None and world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline_prefill(PREFILL[args.workload], PREFILL[args.workload]["seed"])
+            res["cpu_baseline"] = cpu_baseline_prefill(LAYER_WORKLOADS[args.workload],
+                                                       LAYER_WORKLOADS[args.workload]["seed"])
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
         return 0
     res = run_gpu(args, rank, world, local)
     if rank == 0 and res is not None:
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(args.batch, SEED_BASE)
+            res["cpu_baseline"] = cpu_baseline(args.batch, SEED_BASE, one_thread=True)
+            cpu_baselines_for(res.get("workloads", []))
         print(json.dumps(res), flush=True)
     return 0
 

@@ -37,6 +37,13 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const 
                                const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,
                                void* ws, cudaStream_t st);
 
+// INT4 group-128 weight-streaming path (moe_ffn_w4.cu): activation staging, then the
+// persistent TMA-fed gate/up and down GEMVs.  K = H, I <= 8192.
+bool w4_gemv_shape_supported(int64_t H, int64_t I);
+size_t w4_gemv_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
+cudaError_t launch_w4_gemv(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H, int I,
+                           int E, int k, uint16_t* y_rows, void* ws, cudaStream_t st);
+
 // Tensor-core (tcgen05) grouped GEMM path, used by launch_grouped_ffn when the
 // experts see enough rows on average (use_umma_path); W4 group-128 weights.
 bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt);

@@ -352,21 +352,25 @@ size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64
  * from the device): with T*k >= 32*E and W4G128 or NVFP4 weights, a tensor-core GEMM
  * (weights dequantised into tensor memory once per tile of up to 192 routed rows,
  * bf16 operands for W4, fp16 for NVFP4); otherwise a weight-streaming GEMV
- * (dequantisation in registers, weights read once per pass of up to 16 rows).  For
+ * (dequantisation in registers, weights read once per pass of up to 16 rows).  The W4
+ * GEMV stages x once per call as fp16 x/16, streams each expert's weights with bulk
+ * copies through shared memory and turns every nibble into its exact code q = u - 8
+ * before the fp16 tensor-core product; it supports H, I <= 8192.  For
  * BITPLANE8 expert e is read at bits[p] planes for pair p (planes 0..bits[p]-1, floor
  * and compensation as above); expert e's weights are fetched to max_p bits[p].
  *   x bf16 [T][H];  routing: as written by moe_route_topk;  bits uint8 [T*k]
  *   (BITPLANE8 only, values 1..8, else may be NULL);  y_rows bf16 [T*k][H].
  * Requires H % 256 == 0, I % 128 == 0, the limits of moe_route_topk, and workspace
- * >= moe_ffn_workspace_bytes(...) (scratch: h, and for the GEMM path the token rows
- * gathered into routed order; contents need not be initialised).  Not bit-exact: fp32
+ * >= moe_ffn_workspace_bytes(...) (scratch: h; for the W4 GEMV also the staged x; for
+ * the GEMM path the token rows gathered into routed order; contents need not be
+ * initialised).  Not bit-exact: fp32
  * accumulation order, the rounding of h (and, on the GEMM path, of each dequantised
  * W4 weight to bf16) differ from an fp64 reference (ExactMoE: the low-bit layer is
  * not numerically identical to BF16); the FFN tolerance covers both paths.
- * Range: the GEMV stages W4 activations as fp16 x/16 and x/256, and NVFP4 activations
- * and h (both paths) as fp16 * 2^-8, so |x| < 2^20 (W4) and |x|, |h| < 2^24 (NVFP4) keep
- * them finite; magnitudes below 2^-10 (W4) or 2^-6 (NVFP4) fall into fp16's subnormal
- * range (absolute error at most 2^-20 or 2^-16).  Bitplane activations are staged in
+ * Range: the W4 GEMV stages x and h as fp16 x/16 and h/16, and the NVFP4 paths stage
+ * activations and h as fp16 * 2^-8, so |x|, |h| < 2^20 (W4) and |x|, |h| < 2^24 (NVFP4)
+ * keep them finite; magnitudes below 2^-10 (W4) or 2^-6 (NVFP4) fall into fp16's
+ * subnormal range (absolute error at most 2^-20 or 2^-16).  Bitplane activations are staged in
  * bf16 scaled by up to 2^7 (|x| < 2^120). */
 moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
                              const moe_experts_t* experts, const uint8_t* bits,

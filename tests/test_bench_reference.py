@@ -36,6 +36,29 @@ def test_reference_arm_other_ranks_do_no_work():
 
 
 @pytest.mark.parametrize("workload,steps", [("decode", 512), ("bitplane-h2048-e64", 512),
-                                            ("prefill-h2048-e128", 20), ("prefill-h7168-e256", 20)])
+                                            ("prefill-h2048-e128", 20), ("prefill-h7168-e256", 20),
+                                            ("layer-h7168-e256-t64-nvfp4", 200), ("layer-h2048-e64-t16", 200)])
 def test_default_steps_per_workload(workload, steps):
     assert bench.parse_args(["--workload", workload]).steps == steps
+
+
+def test_every_extra_workload_is_defined():
+    # one record per benchmark configuration besides the headline decode stack at batch 8
+    for name in bench.EXTRA_WORKLOADS:
+        assert name == "decode-b1" or name in bench.LAYER_WORKLOADS
+    shapes = {(c["H"], c["I"], c["E"], c.get("fmt", "w4"), c["T"]) for c in bench.LAYER_WORKLOADS.values()}
+    for want in [(2048, 1024, 64, "w4", 16), (2048, 768, 128, "w4", 2048), (2048, 1024, 64, "bitplane", 64),
+                 (7168, 2048, 256, "w4", 1), (7168, 2048, 256, "w4", 64), (7168, 2048, 256, "w4", 4096),
+                 (7168, 2048, 256, "nvfp4", 1), (7168, 2048, 256, "nvfp4", 64), (7168, 2048, 256, "nvfp4", 4096)]:
+        assert want in shapes
+
+
+def test_path_and_bytes_per_workload():
+    c = bench.LAYER_WORKLOADS
+    assert not bench.gemm_path(c["layer-h7168-e256-t64"]) and bench.gemm_path(c["prefill-h7168-e256"])
+    assert bench.gemm_path(c["prefill-h2048-e128"]) and not bench.gemm_path(c["bitplane-h2048-e64"])
+    # W4 g128: half a byte per weight + one bf16 scale per 128 weights (the OLMoE-like expert: 3.244 MB)
+    assert bench.expert_bytes(c["layer-h2048-e64-t16"]) == bench.W4_EXPERT_BYTES == 3244032
+    # NVFP4: half a byte + one E4M3 byte per 16 weights + two fp32 per-tensor scales
+    n = 3 * 7168 * 2048
+    assert bench.expert_bytes(c["layer-h7168-e256-t1-nvfp4"]) == n // 2 + n // 16 + 8

@@ -170,6 +170,8 @@ FFN_CASES = [
     (200, 256, 128, 4, 2),     # ~100 tokens per expert: several 16-token passes
     (16, 2048, 1024, 16, 4),   # OLMoE-like expert shape, decode-sized
     (3, 768, 384, 8, 2),       # K = 768 / 384: uneven split of groups over warps
+    (90, 1024, 256, 4, 1),     # ~22 tokens per expert: two token chunks per weight pass
+    (20, 7168, 384, 3, 1),     # K = 7168: seven weight stages per unit, 56 scale groups
 ]
 
 
