@@ -45,6 +45,7 @@ H, I, E, K_TOP, LAYERS = 2048, 1024, 64, 8, 16
 SEED_BASE = 0x5EED0002
 W4_EXPERT_BYTES = (2 * I * H + H * I) // 2 + (2 * I * (H // 128) + H * (I // 128)) * 2  # packed + bf16 scales
 W13_EXPERT_BYTES = 2 * I * H // 2 + 2 * I * (H // 128) * 2
+W4_GEMV_LAUNCHES = 2  # kernels of one moe_grouped_ffn call on the W4 weight-streaming path
 W2_EXPERT_BYTES = H * I // 2 + H * (I // 128) * 2
 
 # Single-layer workloads (one MoE FFN layer per step on fresh tokens): shapes, routing,
@@ -67,6 +68,9 @@ LAYER_WORKLOADS = {
     "layer-h7168-e256-t1-nvfp4": dict(T=1, fmt="nvfp4", desc=_DSV3_DESC % (_FP4, 1), **_DSV3),
     "layer-h7168-e256-t64-nvfp4": dict(T=64, fmt="nvfp4", desc=_DSV3_DESC % (_FP4, 64), **_DSV3),
     "prefill-h7168-e256-nvfp4": dict(T=4096, fmt="nvfp4", desc=_DSV3_DESC % (_FP4, 4096), **_DSV3),
+    "prefill-h7168-e256-w4a4": dict(T=4096, fmt="nvfp4", act="nvfp4",
+                                    desc=_DSV3_DESC % (_FP4 + " weights and NVFP4 activations quantised on the fly "
+                                                       "(W4A4)", 4096), **_DSV3),
     "bitplane-h2048-e64": dict(T=64, H=2048, I=1024, E=64, k=8, router="normal", zipf=False, seed=0x5EED0004,
                                fmt="bitplane", bits="rule",
                                desc="one MoE FFN layer, H2048 I1024 E64 top-8, 8-bitplane experts, each "
@@ -86,7 +90,8 @@ PREFILL = LAYER_WORKLOADS
 # configuration besides the headline decode stack at batch 8.
 EXTRA_WORKLOADS = ["decode-b1", "layer-h2048-e64-t16", "prefill-h2048-e128", "bitplane-h2048-e64",
                    "bitplane-h2048-e64-duorate", "layer-h7168-e256-t1", "layer-h7168-e256-t64", "prefill-h7168-e256",
-                   "layer-h7168-e256-t1-nvfp4", "layer-h7168-e256-t64-nvfp4", "prefill-h7168-e256-nvfp4"]
+                   "layer-h7168-e256-t1-nvfp4", "layer-h7168-e256-t64-nvfp4", "prefill-h7168-e256-nvfp4",
+                   "prefill-h7168-e256-w4a4"]
 # bitplane experts: bytes of one plane of one expert's w13 + w2, and of their bf16 scales
 BP_PLANE_BYTES = (2 * I * H + H * I) // 8
 BP_SCALE_BYTES = (2 * I * (H // 128) + H * (I // 128)) * 2
@@ -108,6 +113,9 @@ def parse_args(argv=None):
     ap.add_argument("--cache-slots", type=int, default=0,
                     help="decode with each layer's experts in pinned host memory and this many device slots "
                          "per layer (0: every expert resident in HBM)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="single-layer workloads only, for profiling: this many experts instead of the "
+                         "configuration's, with the tokens scaled to keep the rows per expert (not a benchmark line)")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers in the stack (16 is the benchmark workload; fewer only for profiling)")
     args = ap.parse_args(argv)
@@ -293,9 +301,9 @@ class DecodeStack:
     @property
     def kernels_per_step(self):
         # router: one launch for up to 16 tokens whose bf16 rows fit 64 KiB, else logits,
-        # top-k and permutation; then gate/up, down and combine
-        route = 1 if (self.B <= 16 and self.B * H * 2 <= 64 * 1024) else 3
-        return self.L * (route + 3)
+        # top-k and permutation; then the grouped FFN (W4_GEMV_LAUNCHES) and the combine
+        route = 1 if fused_router(self.B, H) else 3
+        return self.L * (route + W4_GEMV_LAUNCHES + 1)
 
 
 class CachedDecodeStack(DecodeStack):
@@ -344,6 +352,10 @@ class CachedDecodeStack(DecodeStack):
         moe.moe_combine(self.y_rows, self.rs, self.B, K_TOP, residual=x, out=nxt)
         if log_active:
             self.n_active[l:l + 1].copy_(self.routing.expert_list[:1])
+
+    def step(self, log_active=False):
+        for l in range(self.L):
+            self.layer(l, log_active)
 
     def fetched(self):
         """(bytes copied over the host link, experts served, hits) of the last step, all layers."""
@@ -605,7 +617,9 @@ def expert_bytes(cfg) -> int:
 
 def gemm_path(cfg) -> bool:
     """moe_grouped_ffn's own choice: the tensor-core GEMM for W4 / NVFP4 batches with
-    T*k >= 32*E, else the weight-streaming GEMV."""
+    T*k >= 32*E, else the weight-streaming GEMV (W4A4 always takes the GEMM)."""
+    if cfg.get("act") == "nvfp4":
+        return True
     return cfg.get("fmt") != "bitplane" and cfg["T"] * cfg["k"] >= 32 * cfg["E"]
 
 
@@ -658,8 +672,10 @@ class PrefillLayer:
             if cfg["zipf"] else None
         self.routing = moe.Routing.empty(T, Ee, k, device)
         self.route_ws = moe.moe_route_workspace(T, Ee, k, device)
-        self.ffn_ws = torch.empty(max(moe.moe_ffn_workspace_bytes(T, Hh, Ii, Ee, k, self.fmt), 16),
-                                  dtype=torch.uint8, device=device)
+        self.w4a4 = cfg.get("act") == "nvfp4"
+        ws_bytes = (moe.moe_ffn_w4a4_workspace_bytes(T, Hh, Ii, Ee, k) if self.w4a4
+                    else moe.moe_ffn_workspace_bytes(T, Hh, Ii, Ee, k, self.fmt))
+        self.ffn_ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
         self.y_rows = torch.empty((T * k, Hh), **bf)
         self.x = torch.empty((T, Hh), **bf)
         self.out = torch.empty((T, Hh), **bf)
@@ -727,8 +743,12 @@ class PrefillLayer:
                 moe.moe_expand_bits(self.routing.topk_ids, self.bits_e, c["k"], bits=self.bits)
         if self.ffn_events is not None:
             self.ffn_events[0].record()
-        moe.moe_grouped_ffn(self.x, self.routing, self.copies[copy], c["I"], c["E"], c["k"], y_rows=self.y_rows,
-                            workspace=self.ffn_ws, bits=self.bits)
+        if self.w4a4:
+            moe.moe_grouped_ffn_w4a4(self.x, self.routing, self.copies[copy], c["I"], c["E"], c["k"],
+                                     y_rows=self.y_rows, workspace=self.ffn_ws)
+        else:
+            moe.moe_grouped_ffn(self.x, self.routing, self.copies[copy], c["I"], c["E"], c["k"], y_rows=self.y_rows,
+                                workspace=self.ffn_ws, bits=self.bits)
         if self.ffn_events is not None:
             self.ffn_events[1].record()
         moe.moe_combine(self.y_rows, self.routing, c["T"], c["k"], residual=self.x, out=self.out)
@@ -740,7 +760,10 @@ class PrefillLayer:
         c = self.cfg
         route = 1 if fused_router(c["T"], c["H"]) else 3  # logits + top-k + permutation otherwise
         widths = 1 if self.bits is not None else 0        # select_bits / expand_bits
-        ffn = 3 if gemm_path(c) else 2                    # (row gather +) gate/up + down
+        if self.w4a4:  # x: amax, codes, routed exact values; gate/up; h: codes, exact values; down
+            ffn = 7
+        else:
+            ffn = 3 if gemm_path(c) else W4_GEMV_LAUNCHES if self.fmt == self.moe.FMT_W4G128 else 2
         return route + widths + ffn + 1                   # + combine
 
 
@@ -752,7 +775,12 @@ def run_prefill(args, rank, world, local):
     init_dist(world, "nccl")
     import bit_mixed_precision_router_b200 as moe
     moe.load()
-    rec = bench_layer(moe, torch, device, LAYER_WORKLOADS[args.workload], args.steps, max(args.warmup, 3), rank,
+    cfg = LAYER_WORKLOADS[args.workload]
+    if args.experts:
+        cfg = dict(cfg, E=args.experts, T=max(1, cfg["T"] * args.experts // cfg["E"]),
+                   desc=cfg["desc"] + " -- profiling scale: %d experts, tokens scaled to keep the rows per expert"
+                        % args.experts)
+    rec = bench_layer(moe, torch, device, cfg, args.steps, max(args.warmup, 3), rank,
                       world, local, e2e=not args.no_e2e)
     if world > 1:
         import torch.distributed as dist
@@ -879,10 +907,11 @@ def bench_layer(moe, torch, device, cfg, K, W, rank, world, local, e2e=True):
         achieved = flops / avg_s / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
                     "frac": round(achieved / bf16_peak, 4),
-                    "peak_kind": peak_kind + " bf16 burst" + (" (the fp16 MMAs of this path have the same dense "
-                                                              "peak)" if cfg.get("fmt") == "nvfp4" else ""),
+                    "peak_kind": peak_kind + " bf16 burst (the fp16 MMAs of this path have the same dense peak)",
                     "traffic": None,
-                    "kernel": "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
+                    "kernel": ("k_ffn_umma gate/up + down with the activation quantisers (one moe_grouped_ffn_w4a4 "
+                               "call; fp16 tensor-core products of the exact NVFP4 values)") if cfg.get("act") else
+                              "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
                     "algorithmic_flops_per_call": flops, "avg_call_us": round(avg_s * 1e6, 1)}
     else:
         achieved = sum(ffn_bytes) / (sum(ffn_ms) / 1e3) / 1e9
@@ -969,7 +998,11 @@ def oracle_prefill_sample(cfg, tokens: int, seed: int):
     else:
         ex = Experts(FMT_BITPLANE8 if bitplane else FMT_W4G128, w13q, w13s, w2q, w2s)
     t0 = time.perf_counter()
-    if bitplane and cfg.get("bits") == "allocated":
+    if cfg.get("act") == "nvfp4":
+        from oracle.w4a4 import w4a4_grouped_ffn
+        r = route(x, wr, bias, k, Ee)
+        combine(w4a4_grouped_ffn(x, r.offsets, r.sorted_pair, k, ex), r.weights, r.pair_to_row, x)
+    elif bitplane and cfg.get("bits") == "allocated":
         # the same per-step path at per-expert widths (every expert at 3 planes, the budget's mean)
         r = route(x, wr, bias, k, Ee)
         y = grouped_ffn(x, r.offsets, r.sorted_pair, k, ex, expand_bits(r.ids, np.full(Ee, 3, np.uint8)))
@@ -1088,7 +1121,7 @@ def cpu_baselines_for(records) -> None:
             r["cpu_baseline"] = cpu_baseline(1, SEED_BASE)
             continue
         cfg = LAYER_WORKLOADS[name]
-        key = (cfg["H"], cfg["I"], cfg["E"], cfg.get("fmt"), cfg.get("bits"), cfg["zipf"], cfg["router"])
+        key = (cfg["H"], cfg["I"], cfg["E"], cfg.get("fmt"), cfg.get("bits"), cfg.get("act"), cfg["zipf"], cfg["router"])
         if key not in shared:
             shared[key] = cpu_baseline_prefill(cfg, cfg["seed"])
             shared[key]["measured_on"] = name

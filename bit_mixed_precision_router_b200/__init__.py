@@ -57,6 +57,7 @@ _SIGS = {
     "moe_quantize_w4g128": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], ctypes.c_int),
     "moe_pack_bitplanes": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], ctypes.c_int),
     "moe_quantize_nvfp4": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moe_quantize_nvfp4_f32": ([_vp, _i64, _i64, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moe_route_workspace_bytes": ([_i64, _i64, _i64], _sz),
     "moe_route_topk": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.POINTER(RoutingT), _vp, _sz, _vp],
                        ctypes.c_int),
@@ -81,6 +82,9 @@ _SIGS = {
     "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
     "moe_grouped_ffn": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
                          _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_ffn_w4a4_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64], _sz),
+    "moe_grouped_ffn_w4a4": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _i64, _i64, _i64, _i64, _i64,
+                              _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_combine": ([_vp, ctypes.POINTER(RoutingT), _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
     "moe_gather_rows": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
     "moe_ids_from_counts": ([_vp, _i64, _i64, _vp, _vp], ctypes.c_int),
@@ -190,6 +194,21 @@ def moe_quantize_nvfp4(w: torch.Tensor, codes=None, block_scales=None, gscale=No
     _check(block_scales, "block_scales", torch.uint8, E * N * (K // 16))
     _check(gscale, "gscale", torch.float32, E)
     _call("moe_quantize_nvfp4", _p(_bits(w)), E, N, K, _p(codes), _p(block_scales), _p(gscale), _stream(stream))
+    return codes, block_scales, gscale
+
+
+def moe_quantize_nvfp4_f32(a: torch.Tensor, codes=None, block_scales=None, gscale=None, stream=None):
+    """fp32 [R][C] as one NVFP4 tensor -> (codes uint8 [R][C/2], block_scales uint8 [R][C/16], gscale fp32 [1])."""
+    R, C = a.shape
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=a.device) if codes is None else codes
+    block_scales = (torch.empty((R, C // 16), dtype=torch.uint8, device=a.device)
+                    if block_scales is None else block_scales)
+    gscale = torch.empty((1,), dtype=torch.float32, device=a.device) if gscale is None else gscale
+    _check(a, "a", torch.float32, R * C)
+    _check(codes, "codes", torch.uint8, R * C // 2)
+    _check(block_scales, "block_scales", torch.uint8, R * C // 16)
+    _check(gscale, "gscale", torch.float32, 1)
+    _call("moe_quantize_nvfp4_f32", _p(a), R, C, _p(codes), _p(block_scales), _p(gscale), _stream(stream))
     return codes, block_scales, gscale
 
 
@@ -534,6 +553,28 @@ def moe_grouped_ffn(x: torch.Tensor, routing: Routing, experts: Experts, I: int,
     rc, ec = routing.c(), experts.c()
     _call("moe_grouped_ffn", _p(_bits(x)), ctypes.byref(rc), ctypes.byref(ec), _p(bits), T, H, I, E, k,
           _p(y_rows), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return y_rows
+
+
+def moe_ffn_w4a4_workspace_bytes(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(load().moe_ffn_w4a4_workspace_bytes(T, H, I, E, k))
+
+
+def moe_grouped_ffn_w4a4(x: torch.Tensor, routing: Routing, experts: Experts, I: int, E: int, k: int,
+                         y_rows: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """The grouped FFN with NVFP4 weights and NVFP4 activations quantised on the fly."""
+    T, H = x.shape
+    y_rows = torch.empty((max(T * k, 1), H), dtype=torch.bfloat16, device=x.device) if y_rows is None else y_rows
+    routing.check(T, E, k)
+    experts.check(H, I, E)
+    _check(y_rows, "y_rows", _BF16, T * k * H)
+    need = moe_ffn_w4a4_workspace_bytes(T, H, I, E, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    rc, ec = routing.c(), experts.c()
+    _call("moe_grouped_ffn_w4a4", _p(_bits(x)), ctypes.byref(rc), ctypes.byref(ec), T, H, I, E, k, _p(y_rows),
+          _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return y_rows
 
 

@@ -113,6 +113,15 @@ moe_status_t moe_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64_t
   return from_cuda(moe::launch_quantize_nvfp4(w, E, N, K, codes, block_scales, gscale, as_stream(stream)));
 }
 
+moe_status_t moe_quantize_nvfp4_f32(const float* a, int64_t R, int64_t C, uint8_t* codes, uint8_t* block_scales,
+                                    float* gscale, moe_stream_t stream) {
+  if (!a || !codes || !block_scales || !gscale) return MOE_ERR_INVALID_ARG;
+  if (R < 1 || C < 1) return MOE_ERR_INVALID_ARG;
+  if (C % 16 != 0 || R > (int64_t(1) << 40) / C) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(a) || !aligned16(codes) || !aligned16(block_scales) || !aligned16(gscale)) return MOE_ERR_MISALIGNED;
+  return from_cuda(moe::launch_quantize_nvfp4_f32(a, R * C, codes, block_scales, gscale, as_stream(stream)));
+}
+
 size_t moe_route_workspace_bytes(int64_t T, int64_t E, int64_t k) {
   if (T < 0 || E < 1 || k < 1) return 0;
   return moe::route_workspace_bytes(T, E, k);
@@ -323,6 +332,35 @@ moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing, co
   if (!moe::device_error_word()) return MOE_ERR_CUDA;
   return from_cuda(moe::launch_grouped_ffn(x, *routing, ex, bits, int(T), int(H), int(I), int(E), int(k), y_rows,
                                            workspace, as_stream(stream)));
+}
+
+size_t moe_ffn_w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
+  if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return 0;
+  return moe::w4a4_workspace_bytes(T, H, I, k);
+}
+
+moe_status_t moe_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t* routing, const moe_experts_t* experts,
+                                  int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, uint16_t* y_rows,
+                                  void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  if (!experts) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  const moe_experts_t& ex = *experts;
+  if (ex.fmt != MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
+  if (!ex.w13 || !ex.w13_scale || !ex.w2 || !ex.w2_scale || !ex.w13_gscale || !ex.w2_gscale) return MOE_ERR_INVALID_ARG;
+  if (H < 256 || H % 256 != 0 || I < 128 || I % 128 != 0 || H > 65536 || I > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (int64_t(E) * 2 * I > INT_MAX || T * k > INT_MAX / (H > I ? H : I)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!x || !y_rows) return MOE_ERR_INVALID_ARG;
+  if ((s = check_routing(routing)) != MOE_OK) return s;
+  const void* ps[] = {x, ex.w13, ex.w13_scale, ex.w2, ex.w2_scale, ex.w13_gscale, ex.w2_gscale, y_rows};
+  for (const void* p : ps)
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < moe::w4a4_workspace_bytes(T, H, I, k)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MOE_ERR_MISALIGNED;
+  if (!moe::device_error_word()) return MOE_ERR_CUDA;
+  return from_cuda(moe::launch_grouped_ffn_w4a4(x, *routing, ex, int(T), int(H), int(I), int(E), int(k), y_rows,
+                                                workspace, as_stream(stream)));
 }
 
 moe_status_t moe_combine(const uint16_t* y_rows, const moe_routing_t* routing, const uint16_t* residual,

@@ -695,7 +695,6 @@ static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
 size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, moe_format_t fmt) {
   if (use_umma_path(T, E, k, fmt)) return umma_workspace_bytes(T, H, I, k);
-  if (fmt == MOE_FMT_W4G128) return w4_gemv_workspace_bytes(T, H, I, k);
   return align256(size_t(T * k * I * 2));  // h
 }
 
@@ -782,7 +781,6 @@ static cudaError_t launch_fmt(const uint16_t* x, const moe_routing_t& r, const m
 }
 
 bool ffn_shape_supported(int64_t H, int64_t I, moe_format_t fmt) {
-  if (fmt == MOE_FMT_W4G128) return w4_gemv_shape_supported(H, I);
   FfnArgs a{};
   bool ok = true;
   for (int64_t K : {H, I}) {
@@ -800,7 +798,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const 
   if (use_umma_path(T, E, k, ex.fmt)) return launch_grouped_ffn_umma(x, r, ex, T, H, I, E, k, y_rows, ws, st);
   switch (ex.fmt) {
     case MOE_FMT_W4G128:
-      return launch_w4_gemv(x, r, ex, T, H, I, E, k, y_rows, ws, st);
+      return launch_fmt<MOE_FMT_W4G128>(x, r, ex, bits, T, H, I, E, k, y_rows, ws, st);
     case MOE_FMT_BITPLANE8:
       return launch_fmt<MOE_FMT_BITPLANE8>(x, r, ex, bits, T, H, I, E, k, y_rows, ws, st);
     case MOE_FMT_NVFP4:

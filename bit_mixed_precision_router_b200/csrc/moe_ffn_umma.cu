@@ -2,7 +2,7 @@
 // (tcgen05, accumulators in tensor memory).
 //
 // Per expert e, the routed rows r in [off_e, off_{e+1}) (sorted order) are
-//   gate/up:  g, u = x[token(r)] . deq(W13_e)^T,  h[r] = silu(g) * u   (bf16)
+//   gate/up:  g, u = x[token(r)] . deq(W13_e)^T,  h[r] = silu(g) * u   (fp16, scaled)
 //   down:     y[r] = h[r] . deq(W2_e)^T                                 (bf16)
 // i.e. the same contraction as the weight-streaming GEMV, organised as a GEMM
 // when each expert sees enough rows for the weights to be worth reusing.
@@ -14,18 +14,18 @@
 // with one lane exchange.
 // Roles inside one persistent CTA (one per SM, 512 threads):
 //   warp  0     TMA producer: per 128-wide K stage (one scale group), the packed
-//               weight tile (8 KiB) into a 4-stage ring and the routed rows (bf16,
+//               weight tile (8 KiB) into a 4-stage ring and the routed rows (fp16,
 //               128-byte swizzled K-major, two 2-D boxes of 64 K) into a 3-stage ring.
 //               For gate/up the rows are the tokens gathered into routed order by
 //               k_gather_rows first (one bandwidth-bound pass; gathering 4 rows per TMA
 //               instruction inside the GEMM could not feed the tensor cores);
 //   warp  1     allocates tensor memory; one thread issues tcgen05.mma (kind::f16,
-//               bf16 in, fp32 accumulate), eight per stage, A from tensor memory, B
+//               fp16 in, fp32 accumulate), eight per stage, A from tensor memory, B
 //               from shared memory; tcgen05.commit releases the stages;
 //   warps 4-11  dequantise the weights from shared memory straight into tensor
 //               memory (tcgen05.st, 2 stages of 64 columns): warp 4 + 4 s + q handles
 //               rows 32 q .. 32 q + 31 of the stages n with n % 2 == s, so two warps
-//               per sub-partition overlap each other's waits; the bf16 weight operand
+//               per sub-partition overlap each other's waits; the fp16 weight operand
 //               never exists in shared memory;
 //   warps 12-15 drain one of the two accumulators (tcgen05.ld) while the other is
 //               being accumulated, apply SwiGLU, and store bf16 rows.
@@ -33,10 +33,12 @@
 // routing offsets and walked round-robin across CTAs.
 //
 // Dequantisation (W4 group-128): (u - 8) * s with u the stored nibble and s the
-// group's bf16 scale, formed as bf16 (128 + u) by byte permutes, then a bf16 add
-// of -136 (exact) and a bf16 multiply by s, rounded once.  That rounding is the
-// only difference from the fp32 dequantisation of the definition (relative 2^-9
-// per weight, inside the FFN tolerance).
+// group's bf16 scale, formed as fp16 (1024 + u) by byte permutes, then an fp16 add of
+// -1032 (exact) and an fp16 multiply by s.  q has 4 significant bits and s 8, so the
+// product needs at most 12: rounded to fp16's 11 it is off by at most 2^-12 relative
+// (exact in most cases), the only difference from the dequantisation of the definition
+// for scales in fp16's normal range (s >= 2^-14).  The activations are the fp16 operand
+// x/16 (h/16 for the down GEMM); the factor 16 is applied in the epilogue.
 //
 // Every wait is bounded (mbar_wait): a wait that runs out sets the device error
 // word and the role stops; the CTA still frees its tensor memory.
@@ -95,9 +97,15 @@ struct UmmaArgs {
   const uint16_t* s;         // W4: bf16 scales [E][n_rows][K/128]
   const uint8_t* bs;         // NVFP4: E4M3 block scales [E][n_rows][K/16]
   const float* gs;           // NVFP4: per-expert fp32 scale of this matrix [E]
-  uint16_t* out;             // gate/up: h [P][I] (bf16; NVFP4: fp16 h/256); down: y [P][H] bf16
+  uint16_t* out;             // gate/up: h [P][I] (fp16 h/16 for W4, h/256 for NVFP4); down: y [P][H] bf16
   int out_ld;
   unsigned* err;
+  // NVFP4 activations (W4A4): the B operand holds the exact values e2m1 * e4m3 of the
+  // quantised activations, whose tensor's amax is *act_amax (scale amax / 2688); gate/up
+  // then writes h as fp32 to out_f32 and its amax to *out_amax (the next quantisation)
+  const float* act_amax;
+  float* out_f32;
+  float* out_amax;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -192,35 +200,37 @@ MOE_DEVICE uint64_t sw128_desc(uint32_t saddr) {
   d |= uint64_t(2) << 61;             // 128-byte swizzle
   return d;
 }
-// Instruction descriptor: fp32 accumulate, A and B both bf16 (W4) or both fp16 (NVFP4),
-// both K-major, M = 128.
+// Instruction descriptor: fp32 accumulate, A and B both fp16 (both formats), both
+// K-major, M = 128.
 template <int FMT>
 MOE_DEVICE uint32_t idesc_mma(int n) {
-  const uint32_t ab = (FMT == MOE_FMT_NVFP4) ? 0u : 1u;  // 0 = f16, 1 = bf16
+  constexpr uint32_t ab = 0u;  // 0 = f16 (1 would be bf16)
   return (1u << 4) | (ab << 7) | (ab << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTM >> 4) << 24);
+}
+// The activation operand's scale: W4 stages x/16 and h/16, NVFP4 x/256 and h/256.
+template <int FMT>
+__host__ __device__ constexpr float act_scale() {
+  return FMT == MOE_FMT_NVFP4 ? 1.f / 256.f : 1.f / 16.f;
 }
 
 // ---------------------------------------------------------------- W4 dequant
 // w holds elements 8i..8i+7 of one row (element j at bits 4j); p[0..3] receive
-// the pairs (0,1), (2,3), (4,5), (6,7) as bf16x2 (128 + u_lo, 128 + u_hi).
+// the pairs (0,1), (2,3), (4,5), (6,7) as fp16x2 (1024 + u_lo, 1024 + u_hi).
 MOE_DEVICE void w4_word_pairs(uint32_t w, uint32_t (&p)[4]) {
   const uint32_t lo = w & 0x0F0F0F0Fu;         // n0 n2 n4 n6
   const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // n1 n3 n5 n7
   const uint32_t u01 = __byte_perm(lo, hi, 0x5140);  // n0 n1 n2 n3
   const uint32_t u23 = __byte_perm(lo, hi, 0x7362);  // n4 n5 n6 n7
-  const uint32_t k43 = 0x43434343u;
-  p[0] = __byte_perm(u01, k43, 0x4140);
-  p[1] = __byte_perm(u01, k43, 0x4342);
-  p[2] = __byte_perm(u23, k43, 0x4140);
-  p[3] = __byte_perm(u23, k43, 0x4342);
+  const uint32_t k64 = 0x64646464u;  // high byte of fp16 1024
+  p[0] = __byte_perm(u01, k64, 0x4140);
+  p[1] = __byte_perm(u01, k64, 0x4342);
+  p[2] = __byte_perm(u23, k64, 0x4140);
+  p[3] = __byte_perm(u23, k64, 0x4342);
 }
-MOE_DEVICE uint32_t bf16x2_add(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hadd2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-MOE_DEVICE uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
+MOE_DEVICE uint32_t hadd2u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 // ---------------------------------------------------------------- work list
@@ -468,7 +478,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
                 v[h][4 * i + j] = hmul2(e2m1x2_to_h2((words[i] >> (8 * j)) & 0xFFu), sb2[4 * h + (i >> 1)]);
           }
         } else {
-          const uint32_t s2 = sv.x | (sv.x << 16);
+          const __half sh = __float2half_rn(bf16_bits_to_float(uint16_t(sv.x)));  // exact in fp16's normal range
+          const uint32_t s2 = uint32_t(__half_as_ushort(sh)) * 0x10001u;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t words[8] = {wq[2 * h].x,     wq[2 * h].y,     wq[2 * h].z,     wq[2 * h].w,
@@ -478,7 +489,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
               uint32_t p[4];
               w4_word_pairs(words[i], p);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) v[h][4 * i + j] = bf16x2_mul(bf16x2_add(p[j], 0xC308C308u), s2);  // (u-8)*s
+              for (int j = 0; j < 4; ++j) v[h][4 * i + j] = hmul2(hadd2u(p[j], 0xE408E408u), s2);  // (u-8)*s
             }
           }
         }
@@ -505,8 +516,12 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       const int ab = it & 1;
       if (!warp_wait(&accFull[ab], (it >> 1) & 1, a.err)) break;
       tc_fence_after();
-      // NVFP4: the accumulator holds sum (e2m1 * e4m3) * x / 256
-      const float post = (FMT == MOE_FMT_NVFP4) ? 256.f * a.gs[tl.e] : 1.f;
+      // the accumulator holds sum w' * x * act_scale (NVFP4: w' = e2m1 * e4m3, the
+      // per-tensor scale still to apply; W4A4: sum w' * a' with a' = e2m1 * e4m3 of the
+      // activations, both per-tensor scales still to apply)
+      float post = (FMT == MOE_FMT_NVFP4) ? 256.f * a.gs[tl.e] : 16.f;
+      if (FMT == MOE_FMT_NVFP4 && a.act_amax) post = a.gs[tl.e] * __fdiv_rn(*a.act_amax, 2688.0f);
+      float amax = 0.f;
       for (int c0 = 0; c0 < tl.nrows; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + uint32_t(ab * kTN + c0), v);
@@ -526,11 +541,20 @@ __global__ void __launch_bounds__(kThreadsU, 1)
             const float up = __shfl_xor_sync(0xffffffffu, mine, 16);
             if (lane < 16 && c < nc) {
               const float hv = silu(mine) * up;
-              o[size_t(c) * a.out_ld] = (FMT == MOE_FMT_NVFP4) ? __half_as_ushort(__float2half_rn(hv * (1.f / 256.f)))
-                                                                : float_to_bf16_bits(hv);
+              if (a.out_f32) {
+                a.out_f32[size_t(tl.r0 + c0 + c) * a.out_ld + tl.wt * 64 + quarter * 16 + lane] = hv;
+                amax = fmaxf(amax, fabsf(hv));
+              } else {
+                o[size_t(c) * a.out_ld] = __half_as_ushort(__float2half_rn(hv * act_scale<FMT>()));
+              }
             }
           }
         }
+      }
+      if (MODE == kGateUp && a.out_f32) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) atomicMax(reinterpret_cast<unsigned*>(a.out_amax), __float_as_uint(amax));
       }
       tc_fence_before();
       __syncwarp();
@@ -546,9 +570,9 @@ __global__ void __launch_bounds__(kThreadsU, 1)
   }
 }
 
-// xs[r] = x[sorted_pair[r] / k]: the token rows in routed order; one warp per row,
-// 16 bytes per lane per step, four steps in flight.
-// NVFP4: the rows are written as fp16 x/256 (the GEMM's B operand type).
+// xs[r] = x[sorted_pair[r] / k]: the token rows in routed order, written as the GEMM's
+// fp16 B operand x * act_scale (x/16 for W4, x/256 for NVFP4); one warp per row, 16
+// bytes per lane per step, four steps in flight.
 template <int FMT>
 __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_pair,
                                                      int P, int k, int row16, uint4* __restrict__ xs) {
@@ -568,22 +592,44 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x
       for (int u = 0; u < 4; ++u) {
         const int c = c0 + 32 * u + lane;
         if (c < row16) {
-          if (FMT == MOE_FMT_NVFP4) {
-            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            uint32_t o[4];
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          uint32_t o[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const __half2 hh = __floats2half2_rn(bf16_lo(w[i]) * (1.f / 256.f), bf16_hi(w[i]) * (1.f / 256.f));
-              o[i] = *reinterpret_cast<const uint32_t*>(&hh);
-            }
-            dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
-          } else {
-            dst[c] = v[u];
+          for (int i = 0; i < 4; ++i) {
+            const __half2 hh =
+                __floats2half2_rn(bf16_lo(w[i]) * act_scale<FMT>(), bf16_hi(w[i]) * act_scale<FMT>());
+            o[i] = *reinterpret_cast<const uint32_t*>(&hh);
           }
+          dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
     }
   }
+}
+
+// B operand of the W4A4 GEMMs: row r of dst = the exact fp16 values e2m1 * e4m3 of the
+// NVFP4 activation row src(r) (gate/up: the token of routed row r; down: r itself).  One
+// thread per block of 16 elements (8 code bytes, one E4M3 scale -> 32 bytes of fp16).
+__global__ void __launch_bounds__(256) k_dequant_rows_nvfp4(const uint8_t* __restrict__ codes,
+                                                            const uint8_t* __restrict__ sb,
+                                                            const int32_t* __restrict__ sorted_pair, int k,
+                                                            int64_t nblocks, int C16, uint4* __restrict__ dst) {
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= nblocks) return;
+  const int64_t r = i / C16;
+  const int b = int(i - r * C16);
+  const int64_t src = sorted_pair ? int64_t(__ldg(sorted_pair + r) / k) : r;
+  const int64_t blk = src * C16 + b;
+  const uint2 cw = *reinterpret_cast<const uint2*>(codes + blk * 8);
+  const uint32_t s2 = e4m3_to_h2(sb[blk]);
+  uint32_t o[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o[j] = hmul2(e2m1x2_to_h2((cw.x >> (8 * j)) & 0xFFu), s2);
+    o[4 + j] = hmul2(e2m1x2_to_h2((cw.y >> (8 * j)) & 0xFFu), s2);
+  }
+  dst[i * 2] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[i * 2 + 1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // ---------------------------------------------------------------- host side
@@ -656,7 +702,7 @@ bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt) {
 
 static size_t align256u(size_t b) { return (b + 255) / 256 * 256; }
 size_t umma_h_bytes(int64_t T, int64_t I, int64_t k) { return align256u(size_t(T * k * I * 2)); }
-// h [P][I], then the routed token rows [P][H] (2-byte elements: bf16 for W4, fp16/256 for NVFP4)
+// h [P][I], then the routed token rows [P][H] (fp16: x/16 for W4, x/256 for NVFP4)
 size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k) {
   return umma_h_bytes(T, I, k) + align256u(size_t(T * k * H * 2));
 }
@@ -675,8 +721,7 @@ static cudaError_t launch_umma_fmt(const uint16_t* x, const moe_routing_t& r, co
   if (!a.err) return cudaErrorInvalidDevice;
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  const CUtensorMapDataType act_type =
-      (FMT == MOE_FMT_NVFP4) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType act_type = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   // the token rows in routed order, after h in the workspace
   uint16_t* xs = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(hbuf) + umma_h_bytes(T, I, k));
   k_gather_rows<FMT><<<4 * nsm, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), r.sorted_pair, P, k, H / 8,
@@ -724,6 +769,105 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
     return launch_umma_fmt<MOE_FMT_W4G128>(x, r, ex, T, H, I, E, k, y_rows, hbuf, st);
   if (ex.fmt == MOE_FMT_NVFP4) return launch_umma_fmt<MOE_FMT_NVFP4>(x, r, ex, T, H, I, E, k, y_rows, hbuf, st);
   return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------- W4A4 (NVFP4 activations)
+// Workspace: two amax words, x codes [T][H/2] and scales [T][H/16], the routed B rows
+// fp16 [P][H], h fp32 [P][I], h codes [P][I/2] and scales [P][I/16], h B rows fp16 [P][I].
+struct W4a4Plan {
+  size_t amax, xc, xsb, bx, hf, hc, hsb, bh, total;
+};
+static W4a4Plan w4a4_plan(int64_t T, int64_t H, int64_t I, int64_t k) {
+  const int64_t P = T * k;
+  W4a4Plan p{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += align256u(bytes);
+    return at;
+  };
+  p.amax = take(256);
+  p.xc = take(size_t(T * H / 2));
+  p.xsb = take(size_t(T * H / 16));
+  p.bx = take(size_t(P * H * 2));
+  p.hf = take(size_t(P * I * 4));
+  p.hc = take(size_t(P * I / 2));
+  p.hsb = take(size_t(P * I / 16));
+  p.bh = take(size_t(P * I * 2));
+  p.total = o;
+  return p;
+}
+
+size_t w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k) { return w4a4_plan(T, H, I, k).total; }
+
+cudaError_t launch_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H,
+                                    int I, int E, int k, uint16_t* y_rows, void* ws, cudaStream_t st) {
+  const int P = T * k;
+  const W4a4Plan pl = w4a4_plan(T, H, I, k);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* amax_x = reinterpret_cast<float*>(base + pl.amax);
+  float* amax_h = amax_x + 1;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  // x -> NVFP4 (one tensor), then its exact values in routed-row order
+  cudaError_t err = launch_act_nvfp4<uint16_t>(x, int64_t(T) * H, base + pl.xc, base + pl.xsb, amax_x, st);
+  if (err != cudaSuccess) return err;
+  int64_t nb = int64_t(P) * (H / 16);
+  k_dequant_rows_nvfp4<<<unsigned((nb + 255) / 256), 256, 0, st>>>(base + pl.xc, base + pl.xsb, r.sorted_pair, k, nb,
+                                                                   H / 16, reinterpret_cast<uint4*>(base + pl.bx));
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if ((err = cudaMemsetAsync(amax_h, 0, sizeof(float), st)) != cudaSuccess) return err;
+  UmmaArgs a{};
+  a.E = E;
+  a.k = k;
+  a.I = I;
+  a.offsets = r.expert_offsets;
+  a.sorted_pair = r.sorted_pair;
+  a.err = device_error_word();
+  if (!a.err) return cudaErrorInvalidDevice;
+  CUtensorMap tb, tw;
+  // gate/up: B = the routed rows of x's exact values, h written as fp32 with its amax
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + pl.bx, uint64_t(H), uint64_t(P), uint64_t(H) * 2,
+                   kAtomK, kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w13, uint64_t(H) / 2, uint64_t(E) * 2 * I,
+                   uint64_t(H) / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  a.K = H;
+  a.n_rows = 2 * I;
+  a.wtiles = I / 64;
+  a.bs = static_cast<const uint8_t*>(ex.w13_scale);
+  a.gs = ex.w13_gscale;
+  a.out = nullptr;
+  a.out_ld = I;
+  a.act_amax = amax_x;
+  a.out_f32 = reinterpret_cast<float*>(base + pl.hf);
+  a.out_amax = amax_h;
+  err = launch_umma_one<MOE_FMT_NVFP4, kGateUp>(tb, tw, a, st);
+  if (err != cudaSuccess) return err;
+  // h (fp32, its amax already taken by the epilogue) -> NVFP4, exact values as the down B
+  nb = int64_t(P) * (I / 16);
+  err = launch_act_nvfp4_codes<float>(reinterpret_cast<const float*>(base + pl.hf), int64_t(P) * I, base + pl.hc,
+                                      base + pl.hsb, amax_h, st);
+  if (err != cudaSuccess) return err;
+  k_dequant_rows_nvfp4<<<unsigned((nb + 255) / 256), 256, 0, st>>>(base + pl.hc, base + pl.hsb, nullptr, 1, nb,
+                                                                   I / 16, reinterpret_cast<uint4*>(base + pl.bh));
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + pl.bh, uint64_t(I), uint64_t(P), uint64_t(I) * 2,
+                   kAtomK, kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 64,
+                   kTM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  a.K = I;
+  a.n_rows = H;
+  a.wtiles = H / kTM;
+  a.bs = static_cast<const uint8_t*>(ex.w2_scale);
+  a.gs = ex.w2_gscale;
+  a.out = y_rows;
+  a.out_ld = H;
+  a.act_amax = amax_h;
+  a.out_f32 = nullptr;
+  a.out_amax = nullptr;
+  return launch_umma_one<MOE_FMT_NVFP4, kDown>(tb, tw, a, st);
 }
 
 }  // namespace moe

@@ -37,13 +37,6 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const 
                                const uint8_t* bits, int T, int H, int I, int E, int k, uint16_t* y_rows,
                                void* ws, cudaStream_t st);
 
-// INT4 group-128 weight-streaming path (moe_ffn_w4.cu): activation staging, then the
-// persistent TMA-fed gate/up and down GEMVs.  K = H, I <= 8192.
-bool w4_gemv_shape_supported(int64_t H, int64_t I);
-size_t w4_gemv_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
-cudaError_t launch_w4_gemv(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H, int I,
-                           int E, int k, uint16_t* y_rows, void* ws, cudaStream_t st);
-
 // Tensor-core (tcgen05) grouped GEMM path, used by launch_grouped_ffn when the
 // experts see enough rows on average (use_umma_path); W4 group-128 weights.
 bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt);
@@ -51,6 +44,22 @@ size_t umma_h_bytes(int64_t T, int64_t I, int64_t k);
 size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
 cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
                                     int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st);
+
+// NVFP4 activations (moe_quant.cu): amax of the tensor into *amax (zeroed first), codes
+// and E4M3 block scales; the _codes form takes an amax already computed.  n % 16 == 0.
+template <typename In>
+cudaError_t launch_act_nvfp4(const In* a, int64_t n, uint8_t* codes, uint8_t* block_scales, float* amax,
+                             cudaStream_t st);
+template <typename In>
+cudaError_t launch_act_nvfp4_codes(const In* a, int64_t n, uint8_t* codes, uint8_t* block_scales, const float* amax,
+                                   cudaStream_t st);
+cudaError_t launch_quantize_nvfp4_f32(const float* a, int64_t n, uint8_t* codes, uint8_t* block_scales,
+                                      float* gscale, cudaStream_t st);
+
+// W4A4 prefill (moe_ffn_umma.cu): NVFP4 weights and NVFP4 activations on the tcgen05 GEMM.
+size_t w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
+cudaError_t launch_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H,
+                                    int I, int E, int k, uint16_t* y_rows, void* ws, cudaStream_t st);
 
 // Budgeted per-expert bit allocation (moe_alloc.cu).
 cudaError_t launch_bitplane_distortion(const uint32_t* planes, const uint16_t* scales, int E, int N, int K,

@@ -102,11 +102,18 @@ __global__ void k_pack_bitplanes(const uint16_t* __restrict__ w, int64_t nchunks
 }
 
 // ---------------------------------------------------------------- NVFP4
-// amax of each expert matrix, accumulated as fp32 bits (non-negative floats order
-// like their bit patterns) into gscale[e], which the caller zeroed.
-__global__ void k_nvfp4_amax(const uint16_t* __restrict__ w, int64_t per_expert, float* __restrict__ gscale) {
+// Eight consecutive elements as fp32: bf16 weights or activations, or fp32 activations.
+MOE_DEVICE void load8(const float* p, float (&f)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+
+// amax of each expert matrix (or activation tensor), accumulated as fp32 bits (non-negative
+// floats order like their bit patterns) into gscale[e], which the caller zeroed.
+template <typename In>
+__global__ void k_nvfp4_amax(const In* __restrict__ w, int64_t per_expert, float* __restrict__ gscale) {
   const int e = blockIdx.y;
-  const uint16_t* base = w + int64_t(e) * per_expert;
+  const In* base = w + int64_t(e) * per_expert;
   float amax = 0.f;
   for (int64_t c = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) * 8; c < per_expert;
        c += int64_t(gridDim.x) * blockDim.x * 8) {
@@ -126,7 +133,8 @@ MOE_DEVICE float e4m3_to_float(uint8_t c) {
 }
 
 // One thread per block of 16 elements.  gscale holds amax here (see k_nvfp4_amax).
-__global__ void k_quant_nvfp4(const uint16_t* __restrict__ w, int64_t nblocks, int64_t blocks_per_expert,
+template <typename In>
+__global__ void k_quant_nvfp4(const In* __restrict__ w, int64_t nblocks, int64_t blocks_per_expert,
                               const float* __restrict__ amax_e, uint8_t* __restrict__ codes,
                               uint8_t* __restrict__ block_scales) {
   const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
@@ -197,13 +205,56 @@ cudaError_t launch_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64
   const int threads = 256;
   int64_t bx = (per_expert / 8 + threads - 1) / threads;
   if (bx > 1024) bx = 1024;
-  k_nvfp4_amax<<<dim3(unsigned(bx), unsigned(E)), threads, 0, st>>>(w, per_expert, gscale);
+  k_nvfp4_amax<uint16_t><<<dim3(unsigned(bx), unsigned(E)), threads, 0, st>>>(w, per_expert, gscale);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t nblocks = E * N * K / 16;
-  k_quant_nvfp4<<<dim3(unsigned((nblocks + threads - 1) / threads)), threads, 0, st>>>(
+  k_quant_nvfp4<uint16_t><<<dim3(unsigned((nblocks + threads - 1) / threads)), threads, 0, st>>>(
       w, nblocks, N * K / 16, gscale, codes, block_scales);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   k_nvfp4_finalize<<<dim3(unsigned((E + 255) / 256)), 256, 0, st>>>(gscale, int(E));
+  return cudaGetLastError();
+}
+
+// Activations in NVFP4 for the W4A4 prefill path (the weights' recipe with the whole
+// tensor as one scale unit): amax of `a` into *amax (zeroed here), then codes and block
+// scales; *amax keeps the amax (the scale g = amax / 2688 is taken where it is used).
+template <typename In>
+cudaError_t launch_act_nvfp4(const In* a, int64_t n, uint8_t* codes, uint8_t* block_scales, float* amax,
+                             cudaStream_t st) {
+  cudaError_t err = cudaMemsetAsync(amax, 0, sizeof(float), st);
+  if (err != cudaSuccess) return err;
+  const int threads = 256;
+  int64_t bx = (n / 8 + threads - 1) / threads;
+  if (bx > 2048) bx = 2048;
+  if (bx < 1) bx = 1;
+  k_nvfp4_amax<In><<<dim3(unsigned(bx), 1u), threads, 0, st>>>(a, n, amax);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int64_t nblocks = n / 16;
+  k_quant_nvfp4<In><<<dim3(unsigned((nblocks + threads - 1) / threads)), threads, 0, st>>>(a, nblocks, nblocks, amax,
+                                                                                           codes, block_scales);
+  return cudaGetLastError();
+}
+template cudaError_t launch_act_nvfp4<uint16_t>(const uint16_t*, int64_t, uint8_t*, uint8_t*, float*, cudaStream_t);
+template cudaError_t launch_act_nvfp4<float>(const float*, int64_t, uint8_t*, uint8_t*, float*, cudaStream_t);
+
+// The codes and block scales only, for a tensor whose amax is already in *amax.
+template <typename In>
+cudaError_t launch_act_nvfp4_codes(const In* a, int64_t n, uint8_t* codes, uint8_t* block_scales, const float* amax,
+                                   cudaStream_t st) {
+  const int threads = 256;
+  const int64_t nblocks = n / 16;
+  k_quant_nvfp4<In><<<dim3(unsigned((nblocks + threads - 1) / threads)), threads, 0, st>>>(a, nblocks, nblocks, amax,
+                                                                                           codes, block_scales);
+  return cudaGetLastError();
+}
+template cudaError_t launch_act_nvfp4_codes<float>(const float*, int64_t, uint8_t*, uint8_t*, const float*,
+                                                   cudaStream_t);
+
+cudaError_t launch_quantize_nvfp4_f32(const float* a, int64_t n, uint8_t* codes, uint8_t* block_scales,
+                                      float* gscale, cudaStream_t st) {
+  const cudaError_t err = launch_act_nvfp4<float>(a, n, codes, block_scales, gscale, st);
+  if (err != cudaSuccess) return err;
+  k_nvfp4_finalize<<<1, 32, 0, st>>>(gscale, 1);
   return cudaGetLastError();
 }
 

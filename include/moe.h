@@ -147,6 +147,14 @@ moe_status_t moe_quantize_nvfp4(const uint16_t* w, int64_t E, int64_t N, int64_t
                                 uint8_t* codes, uint8_t* block_scales, float* gscale,
                                 moe_stream_t stream);
 
+/* NVFP4 quantisation of one fp32 tensor as a single scale unit (the activations of the
+ * W4A4 prefill path [MoET: NVFP4]; same recipe as moe_quantize_nvfp4, with the whole
+ * [R][C] tensor in place of one expert matrix).  a fp32 [R][C]; codes uint8 [R][C/2];
+ * block_scales uint8 E4M3 [R][C/16]; gscale fp32 [1] (amax / 2688, also scratch).
+ * Requires C % 16 == 0.  Bit-exact. */
+moe_status_t moe_quantize_nvfp4_f32(const float* a, int64_t R, int64_t C, uint8_t* codes, uint8_t* block_scales,
+                                    float* gscale, moe_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * One layer step: route -> (select_bits) -> grouped_ffn -> combine
  * ------------------------------------------------------------------------ */
@@ -350,33 +358,50 @@ size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64
  *   h = bf16(silu(g) * u),  y_rows[r] = bf16(h . deq(W2_e)^T).
  * Two execution paths, chosen on the host from the shape alone (nothing is read back
  * from the device): with T*k >= 32*E and W4G128 or NVFP4 weights, a tensor-core GEMM
- * (weights dequantised into tensor memory once per tile of up to 192 routed rows,
- * bf16 operands for W4, fp16 for NVFP4); otherwise a weight-streaming GEMV
- * (dequantisation in registers, weights read once per pass of up to 16 rows).  The W4
- * GEMV stages x once per call as fp16 x/16, streams each expert's weights with bulk
- * copies through shared memory and turns every nibble into its exact code q = u - 8
- * before the fp16 tensor-core product; it supports H, I <= 8192.  For
+ * (weights dequantised into tensor memory once per tile of up to 192 routed rows, fp16
+ * operands: W4 weights q*s, NVFP4 weights e2m1*e4m3); otherwise a weight-streaming GEMV
+ * (dequantisation in registers, weights read once per pass of up to 16 rows).  For
  * BITPLANE8 expert e is read at bits[p] planes for pair p (planes 0..bits[p]-1, floor
  * and compensation as above); expert e's weights are fetched to max_p bits[p].
  *   x bf16 [T][H];  routing: as written by moe_route_topk;  bits uint8 [T*k]
  *   (BITPLANE8 only, values 1..8, else may be NULL);  y_rows bf16 [T*k][H].
  * Requires H % 256 == 0, I % 128 == 0, the limits of moe_route_topk, and workspace
- * >= moe_ffn_workspace_bytes(...) (scratch: h; for the W4 GEMV also the staged x; for
- * the GEMM path the token rows gathered into routed order; contents need not be
- * initialised).  Not bit-exact: fp32
+ * >= moe_ffn_workspace_bytes(...) (scratch: h, and for the GEMM path the token rows
+ * gathered into routed order; contents need not be initialised).  Not bit-exact: fp32
  * accumulation order, the rounding of h (and, on the GEMM path, of each dequantised
  * W4 weight to bf16) differ from an fp64 reference (ExactMoE: the low-bit layer is
  * not numerically identical to BF16); the FFN tolerance covers both paths.
- * Range: the W4 GEMV stages x and h as fp16 x/16 and h/16, and the NVFP4 paths stage
- * activations and h as fp16 * 2^-8, so |x|, |h| < 2^20 (W4) and |x|, |h| < 2^24 (NVFP4)
- * keep them finite; magnitudes below 2^-10 (W4) or 2^-6 (NVFP4) fall into fp16's
- * subnormal range (absolute error at most 2^-20 or 2^-16).  Bitplane activations are staged in
+ * Range: the W4 paths stage activations as fp16 x/16 and x/256 (GEMV) or x/16 and h/16
+ * (GEMM), the NVFP4 paths activations and h as fp16 * 2^-8, so |x|, |h| < 2^20 (W4) and
+ * |x|, |h| < 2^24 (NVFP4) keep them finite; magnitudes below 2^-10 (W4) or 2^-6 (NVFP4)
+ * fall into fp16's subnormal range (absolute error at most 2^-20 or 2^-16).  The W4 GEMM
+ * rounds each weight q*s to fp16 (relative 2^-12 at most, for scales >= 2^-14).  Bitplane activations are staged in
  * bf16 scaled by up to 2^7 (|x| < 2^120). */
 moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
                              const moe_experts_t* experts, const uint8_t* bits,
                              int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
                              uint16_t* y_rows, void* workspace, size_t workspace_bytes,
                              moe_stream_t stream);
+
+/* Bytes of device workspace moe_grouped_ffn_w4a4 needs. */
+size_t moe_ffn_w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k);
+
+/* The grouped FFN with NVFP4 weights AND NVFP4 activations (W4A4) for prefill batches
+ * [MoET: NVFP4 for expert GEMMs].  x is quantised on the fly as one tensor by the NVFP4
+ * recipe (E2M1 codes, an E4M3 scale per 16 consecutive elements of a row, one fp32 scale
+ * amax/2688 for the tensor); per expert g, u = x' W13'^T, h = silu(g) u kept in fp32; all
+ * routed rows of h are quantised the same way, as one tensor, from those fp32 values; y_rows
+ * = h' W2'^T (bf16).  Every product is exact: the tensor cores multiply the exact values
+ * e2m1 * e4m3 of both operands (fp16, fp32 accumulation) and the two per-tensor scales
+ * multiply each sum once.  Always the tcgen05 GEMM (any batch size).
+ *   experts: fmt must be MOE_FMT_NVFP4 (as written by moe_quantize_nvfp4); other arguments
+ *   and layouts as for moe_grouped_ffn; workspace >= moe_ffn_w4a4_workspace_bytes(...)
+ *   (scratch: the quantised x and h, their fp16 values in routed order, h in fp32).
+ * Tolerance against the W4A4 definition as for moe_grouped_ffn; an element of h within a
+ * rounding of an E2M1 decision boundary may take the other code (fp32 order). */
+moe_status_t moe_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t* routing, const moe_experts_t* experts,
+                                  int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, uint16_t* y_rows,
+                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* Routing-weighted combine [ExactMoE: the selected experts' outputs weighted by the
  * unchanged routing weights]: out[t] = bf16( sum_{j<k} topk_w[t*k+j] *
