@@ -694,6 +694,9 @@ class PrefillLayer:
         for _ in range(n_copies - 1):
             self.copies.append(moe.Experts(self.fmt, w13[0].clone(), w13[1].clone(), w2[0].clone(), w2[1].clone(),
                                            g(w13[2]), g(w2[2])))
+        if self.w4a4:  # the weight scales in tensor-core order: part of the weights, made untimed
+            for ex in self.copies:
+                ex.w4a4_tiles = moe.moe_w4a4_prepare(ex, Hh, Ii, Ee)
 
     def allocate_widths(self, torch, device, seed):
         """Per-expert widths for the bitplane experts under the read budget: the distortion
@@ -760,10 +763,11 @@ class PrefillLayer:
         c = self.cfg
         route = 1 if fused_router(c["T"], c["H"]) else 3  # logits + top-k + permutation otherwise
         widths = 1 if self.bits is not None else 0        # select_bits / expand_bits
-        if self.w4a4:  # x: amax, codes, routed exact values; gate/up; h: codes, exact values; down
-            ffn = 7
+        if self.w4a4:  # row-tile prefix; x: amax, codes, routed codes + tiled scales; gate/up; h: codes,
+            ffn = 8        # tiled scales; down
         else:
-            ffn = 3 if gemm_path(c) else W4_GEMV_LAUNCHES if self.fmt == self.moe.FMT_W4G128 else 2
+            # GEMM batches: gather, gate/up GEMM + GEMV pass over the small experts, down likewise
+            ffn = 5 if gemm_path(c) else W4_GEMV_LAUNCHES if self.fmt == self.moe.FMT_W4G128 else 2
         return route + widths + ffn + 1                   # + combine
 
 
@@ -902,16 +906,33 @@ def bench_layer(moe, torch, device, cfg, K, W, rank, world, local, e2e=True):
     layer.ffn_events = None
     hbm, bf16_peak, peak_kind = measured_peaks()
     avg_s = statistics.mean(ffn_ms) / 1e3
-    if gemm:
+    if gemm and cfg.get("act"):
+        # W4A4 on the FP4 tensor cores: 2 P 3 H I flops against 4x the bf16 peak (the nominal
+        # fp4 : bf16 ratio) take less time than its bytes at the HBM peak, so HBM bounds it.
+        # Algorithmic bytes: the routed experts' codes and scales, x (bf16), y_rows (bf16),
+        # and h as NVFP4 written and read.
+        flops = 2.0 * T * k * 3 * Hh * Ii
+        nbytes = (statistics.mean(ffn_bytes) - act_bytes + T * Hh * 2 + T * k * Hh * 2
+                  + 2 * T * k * Ii * 9 / 16)
+        achieved = nbytes / avg_s / 1e9
+        fp4_peak = 4.0 * bf16_peak
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4), "peak_kind": peak_kind + " HBM copy", "traffic": None,
+                    "kernel": ("k_ffn_fp4 gate/up + down (block-scaled tcgen05 FP4 MMA) with the activation "
+                               "quantisers (one moe_grouped_ffn_w4a4 call)"),
+                    "algorithmic_bytes_per_call": round(nbytes), "avg_call_us": round(avg_s * 1e6, 1),
+                    "tensor": {"achieved": round(flops / avg_s / 1e12, 1), "peak": round(fp4_peak, 1),
+                               "unit": "TFLOP/s", "frac": round(flops / avg_s / 1e12 / fp4_peak, 4),
+                               "peak_kind": peak_kind + " bf16 burst x 4 (nominal fp4 : bf16 dense ratio)"}}
+    elif gemm:
         flops = 2.0 * T * k * 3 * Hh * Ii
         achieved = flops / avg_s / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
                     "frac": round(achieved / bf16_peak, 4),
                     "peak_kind": peak_kind + " bf16 burst (the fp16 MMAs of this path have the same dense peak)",
                     "traffic": None,
-                    "kernel": ("k_ffn_umma gate/up + down with the activation quantisers (one moe_grouped_ffn_w4a4 "
-                               "call; fp16 tensor-core products of the exact NVFP4 values)") if cfg.get("act") else
-                              "k_ffn_umma gate/up + down with the row gather (one moe_grouped_ffn call)",
+                    "kernel": "k_ffn_umma gate/up + down with the row gather and the GEMV pass over small experts "
+                              "(one moe_grouped_ffn call)",
                     "algorithmic_flops_per_call": flops, "avg_call_us": round(avg_s * 1e6, 1)}
     else:
         achieved = sum(ffn_bytes) / (sum(ffn_ms) / 1e3) / 1e9
@@ -935,7 +956,7 @@ def bench_layer(moe, torch, device, cfg, K, W, rank, world, local, e2e=True):
     else:
         l2 = "no flush: the %.1f GB of expert weights exceed 4 x the 126 MB L2" % (Ee * expert_bytes(cfg) / 1e9)
     rec = {"value": round(value, 1), "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
-           "dtype": "fp16" if fmt == "nvfp4" and gemm else "bf16",
+           "dtype": ("e2m1" if cfg.get("act") else "fp16") if fmt == "nvfp4" and gemm else "bf16",
            "data": "synthetic (seeded Irwin-Hall N(0,1) activations, N(0,0.02) bf16 weights quantised to "
                    + {"nvfp4": "NVFP4", "bitplane": "8 bitplanes"}.get(fmt, "W4A16 g128") + ")",
            "config": {"workload": cfg["desc"], "tokens": T, "hidden": Hh, "intermediate": Ii, "experts": Ee,

@@ -11,7 +11,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import torch
 
@@ -82,9 +82,11 @@ _SIGS = {
     "moe_ffn_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64, ctypes.c_int], _sz),
     "moe_grouped_ffn": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
                          _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_w4a4_scale_tiles_bytes": ([_i64, _i64, _i64], _sz),
+    "moe_w4a4_prepare": ([ctypes.POINTER(ExpertsT), _i64, _i64, _i64, _vp, _sz, _vp], ctypes.c_int),
     "moe_ffn_w4a4_workspace_bytes": ([_i64, _i64, _i64, _i64, _i64], _sz),
-    "moe_grouped_ffn_w4a4": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _i64, _i64, _i64, _i64, _i64,
-                              _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_grouped_ffn_w4a4": ([_vp, ctypes.POINTER(RoutingT), ctypes.POINTER(ExpertsT), _vp, _i64, _i64, _i64, _i64,
+                              _i64, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_combine": ([_vp, ctypes.POINTER(RoutingT), _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
     "moe_gather_rows": ([_vp, _vp, _i64, _i64, _i64, _vp, _vp], ctypes.c_int),
     "moe_ids_from_counts": ([_vp, _i64, _i64, _vp, _vp], ctypes.c_int),
@@ -417,6 +419,8 @@ class Experts:
     w2_scale: torch.Tensor
     w13_gscale: torch.Tensor | None = None
     w2_gscale: torch.Tensor | None = None
+    # NVFP4: the weight-scale tiles of the W4A4 path (moe_w4a4_prepare), made on first use
+    w4a4_tiles: torch.Tensor | None = field(default=None, repr=False)
 
     def c(self) -> ExpertsT:
         return ExpertsT(self.fmt, _p(self.w13), _p(self.w13_scale), _p(self.w2), _p(self.w2_scale),
@@ -556,25 +560,48 @@ def moe_grouped_ffn(x: torch.Tensor, routing: Routing, experts: Experts, I: int,
     return y_rows
 
 
+def moe_w4a4_scale_tiles_bytes(H: int, I: int, E: int) -> int:
+    return int(load().moe_w4a4_scale_tiles_bytes(H, I, E))
+
+
+def moe_w4a4_prepare(experts: Experts, H: int, I: int, E: int, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """The weight scales of NVFP4 experts in the order the FP4 tensor cores read them (once per
+    set of experts; again after the weights change)."""
+    experts.check(H, I, E)
+    need = moe_w4a4_scale_tiles_bytes(H, I, E)
+    out = torch.empty(max(need, 16), dtype=torch.uint8, device=experts.w13.device) if out is None else out
+    ec = experts.c()
+    _call("moe_w4a4_prepare", ctypes.byref(ec), H, I, E, _p(out), out.numel() * out.element_size(), _stream(stream))
+    return out
+
+
 def moe_ffn_w4a4_workspace_bytes(T: int, H: int, I: int, E: int, k: int) -> int:
     return int(load().moe_ffn_w4a4_workspace_bytes(T, H, I, E, k))
 
 
 def moe_grouped_ffn_w4a4(x: torch.Tensor, routing: Routing, experts: Experts, I: int, E: int, k: int,
                          y_rows: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                         stream=None) -> torch.Tensor:
-    """The grouped FFN with NVFP4 weights and NVFP4 activations quantised on the fly."""
+                         stream=None, scale_tiles: torch.Tensor | None = None) -> torch.Tensor:
+    """The grouped FFN with NVFP4 weights and NVFP4 activations quantised on the fly.
+    scale_tiles: moe_w4a4_prepare's output for these experts; if None, the experts' own
+    (prepared on first use and kept in experts.w4a4_tiles)."""
     T, H = x.shape
     y_rows = torch.empty((max(T * k, 1), H), dtype=torch.bfloat16, device=x.device) if y_rows is None else y_rows
     routing.check(T, E, k)
     experts.check(H, I, E)
     _check(y_rows, "y_rows", _BF16, T * k * H)
+    if scale_tiles is None:
+        if experts.w4a4_tiles is None:
+            experts.w4a4_tiles = moe_w4a4_prepare(experts, H, I, E, stream=stream)
+        scale_tiles = experts.w4a4_tiles
+    _check(scale_tiles, "scale_tiles", torch.uint8, moe_w4a4_scale_tiles_bytes(H, I, E))
     need = moe_ffn_w4a4_workspace_bytes(T, H, I, E, k)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
     rc, ec = routing.c(), experts.c()
-    _call("moe_grouped_ffn_w4a4", _p(_bits(x)), ctypes.byref(rc), ctypes.byref(ec), T, H, I, E, k, _p(y_rows),
-          _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _call("moe_grouped_ffn_w4a4", _p(_bits(x)), ctypes.byref(rc), ctypes.byref(ec), _p(scale_tiles), T, H, I, E, k,
+          _p(y_rows), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return y_rows
 
 

@@ -334,33 +334,66 @@ moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing, co
                                            workspace, as_stream(stream)));
 }
 
-size_t moe_ffn_w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
-  if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return 0;
-  return moe::w4a4_workspace_bytes(T, H, I, k);
+// shape rules of the W4A4 path: K stages of 256 elements (H), 64-element K blocks and
+// 64-row gate/up weight tiles (I), 128-row down weight tiles (H)
+static moe_status_t w4a4_shape(int64_t H, int64_t I, int64_t E) {
+  if (H < 256 || H % 256 != 0 || I < 128 || I % 128 != 0 || H > 65536 || I > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (E < 1 || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (int64_t(E) * 2 * I > INT_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
 }
 
-moe_status_t moe_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t* routing, const moe_experts_t* experts,
-                                  int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, uint16_t* y_rows,
-                                  void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+static moe_status_t w4a4_experts(const moe_experts_t* experts) {
   if (!experts) return MOE_ERR_INVALID_ARG;
-  moe_status_t s = check_route_shape(T, E, k);
-  if (s != MOE_OK) return s;
   const moe_experts_t& ex = *experts;
   if (ex.fmt != MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
   if (!ex.w13 || !ex.w13_scale || !ex.w2 || !ex.w2_scale || !ex.w13_gscale || !ex.w2_gscale) return MOE_ERR_INVALID_ARG;
-  if (H < 256 || H % 256 != 0 || I < 128 || I % 128 != 0 || H > 65536 || I > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (int64_t(E) * 2 * I > INT_MAX || T * k > INT_MAX / (H > I ? H : I)) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (T == 0) return MOE_OK;
-  if (!x || !y_rows) return MOE_ERR_INVALID_ARG;
-  if ((s = check_routing(routing)) != MOE_OK) return s;
-  const void* ps[] = {x, ex.w13, ex.w13_scale, ex.w2, ex.w2_scale, ex.w13_gscale, ex.w2_gscale, y_rows};
+  const void* ps[] = {ex.w13, ex.w13_scale, ex.w2, ex.w2_scale, ex.w13_gscale, ex.w2_gscale};
   for (const void* p : ps)
     if (!aligned16(p)) return MOE_ERR_MISALIGNED;
-  if (!workspace || workspace_bytes < moe::w4a4_workspace_bytes(T, H, I, k)) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+size_t moe_w4a4_scale_tiles_bytes(int64_t H, int64_t I, int64_t E) {
+  if (H < 1 || I < 1 || E < 1) return 0;
+  return moe::w4a4_scale_tiles_bytes(H, I, E);
+}
+
+moe_status_t moe_w4a4_prepare(const moe_experts_t* experts, int64_t H, int64_t I, int64_t E, void* scale_tiles,
+                              size_t scale_tiles_bytes, moe_stream_t stream) {
+  moe_status_t s = w4a4_shape(H, I, E);
+  if (s != MOE_OK) return s;
+  if ((s = w4a4_experts(experts)) != MOE_OK) return s;
+  if (!scale_tiles) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(scale_tiles)) return MOE_ERR_MISALIGNED;
+  if (scale_tiles_bytes < moe::w4a4_scale_tiles_bytes(H, I, E)) return MOE_ERR_WORKSPACE;
+  return from_cuda(moe::launch_w4a4_prepare(*experts, int(H), int(I), int(E), static_cast<uint8_t*>(scale_tiles),
+                                            as_stream(stream)));
+}
+
+size_t moe_ffn_w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
+  if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return 0;
+  return moe::w4a4_workspace_bytes(T, H, I, E, k);
+}
+
+moe_status_t moe_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t* routing, const moe_experts_t* experts,
+                                  const void* scale_tiles, int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                                  uint16_t* y_rows, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  moe_status_t s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  if ((s = w4a4_shape(H, I, E)) != MOE_OK) return s;
+  if ((s = w4a4_experts(experts)) != MOE_OK) return s;
+  if (T * k > INT_MAX / (H > I ? H : I)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!x || !y_rows || !scale_tiles) return MOE_ERR_INVALID_ARG;
+  if ((s = check_routing(routing)) != MOE_OK) return s;
+  if (!aligned16(x) || !aligned16(y_rows) || !aligned16(scale_tiles)) return MOE_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < moe::w4a4_workspace_bytes(T, H, I, E, k)) return MOE_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MOE_ERR_MISALIGNED;
   if (!moe::device_error_word()) return MOE_ERR_CUDA;
-  return from_cuda(moe::launch_grouped_ffn_w4a4(x, *routing, ex, int(T), int(H), int(I), int(E), int(k), y_rows,
-                                                workspace, as_stream(stream)));
+  return from_cuda(moe::launch_grouped_ffn_w4a4(x, *routing, *experts, static_cast<const uint8_t*>(scale_tiles),
+                                                int(T), int(H), int(I), int(E), int(k), y_rows, workspace,
+                                                as_stream(stream)));
 }
 
 moe_status_t moe_combine(const uint16_t* y_rows, const moe_routing_t* routing, const uint16_t* residual,

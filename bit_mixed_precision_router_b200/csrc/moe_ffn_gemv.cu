@@ -16,6 +16,9 @@
 // nibble / bit / FP4 -> fp16 or bf16 in registers, mma.sync m16n8k16 with the tokens on N.
 // W4 takes two groups per wait and converts nibbles to fp16 against activations staged
 // in fp16 (see w4h_group).  Expert weights are read from HBM once per token chunk.
+#include <atomic>
+#include <climits>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -24,12 +27,13 @@ namespace moe {
 enum { kGateUp = 0, kDown = 1 };
 constexpr int kRows = 16;     // weight rows per unit
 constexpr int kWarps = 4;     // warps per CTA (W4, NVFP4), each owning whole units
-constexpr int kThreads = 32 * kWarps;
 constexpr int kWarpsBP = 8;   // bitplanes: eight warps share one activation stage
 constexpr int kDepth = 6;     // group steps in flight per warp (NVFP4)
 constexpr int kDepthW4 = 6;   // W4: groups in flight per warp, consumed and refilled two at a time
 constexpr int kMaxTok = 16;   // tokens per activation stage (two n8 tiles)
 constexpr size_t kSmemTarget = 55 * 1024;  // four CTAs per SM
+constexpr int kWarpsWide = 16;                 // wide rows: one 16-warp CTA per SM
+constexpr size_t kSmemTargetWide = 219 * 1024;
 // Bitplanes: a group step holds only the planes the chunk reads (b x 16 rows x 16 bytes),
 // so a fixed per-warp ring of 16 plane slots is min(8, 16 / b) steps deep (8 at b <= 2, 5
 // at b = 3, 4, 3, then 2 at b >= 6); two 8-warp CTAs per SM still stage 16 tokens at
@@ -57,6 +61,7 @@ struct FfnArgs {
   const float* gscale;  // NVFP4
   void* out;            // gate/up: h [P][I]; down: y [P][H]
   int out_ld;
+  int max_rows;  // experts with more routed rows are left to the tensor-core GEMM
   // shared-memory plan (bytes), filled by the launcher
   int nx, x_stride, slot_bytes, warp_bytes, off_x, off_xsum, off_bits;
 };
@@ -403,9 +408,9 @@ MOE_DEVICE void stream_unit_bp(const FfnArgs& a, const uint8_t* wsm, const uint1
 }
 
 // ---------------------------------------------------------------- kernel
-template <int FMT, int MODE>
-__global__ void __launch_bounds__(32 * warps_of<FMT>(), 16 / warps_of<FMT>()) k_ffn_gemv(FfnArgs a) {
-  constexpr int WARPS = warps_of<FMT>(), THREADS = 32 * WARPS;
+template <int FMT, int MODE, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS, 16 / WARPS) k_ffn_gemv(FfnArgs a) {
+  constexpr int THREADS = 32 * WARPS;
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int slot = blockIdx.y;
@@ -413,6 +418,7 @@ __global__ void __launch_bounds__(32 * warps_of<FMT>(), 16 / warps_of<FMT>()) k_
   const int e = a.expert_list[1 + slot];
   const int row0 = a.offsets[e];
   const int n_e = a.offsets[e + 1] - row0;
+  if (n_e > a.max_rows) return;  // this expert's rows go through the tensor-core GEMM
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   const int K = a.K, GK = K / 128;
   const int TPE = (MODE == kGateUp) ? a.I / 8 : a.N / kRows;
@@ -698,21 +704,23 @@ size_t ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k
   return align256(size_t(T * k * I * 2));  // h
 }
 
+// Shared-memory plan of a CTA of `warps` warps within `target` bytes: the warps' rings and
+// scales, then as many staged token rows (nx, at most 16) as fit.
 template <int FMT>
-static bool plan(FfnArgs& a) {
+static bool plan(FfnArgs& a, int warps = warps_of<FMT>(), size_t target = 0) {
   const int K = a.K, GK = K / 128;
   a.slot_bytes = slot_bytes_of<FMT>();
   const int scale_bytes = (FMT == MOE_FMT_NVFP4) ? 0 : int(align256(size_t(kRows) * GK * 2));
   a.warp_bytes = int(align256(size_t(ring_bytes_of<FMT>()) + scale_bytes));
   a.x_stride = stride_16B(K * 2);
   const int nsum = (FMT == MOE_FMT_BITPLANE8) ? 2 : 1;  // bitplanes: X and X'
-  const size_t fixed = size_t(warps_of<FMT>()) * a.warp_bytes + align256(size_t(nsum) * kMaxTok * GK * 4) + 256;
-  const size_t target = (FMT == MOE_FMT_BITPLANE8) ? kSmemTargetBP : kSmemTarget;
+  const size_t fixed = size_t(warps) * a.warp_bytes + align256(size_t(nsum) * kMaxTok * GK * 4) + 256;
+  if (!target) target = (FMT == MOE_FMT_BITPLANE8) ? kSmemTargetBP : kSmemTarget;
   const size_t room = fixed < target ? target - fixed : 0;
   int nx = int(room / size_t(a.x_stride));
   nx = nx < 1 ? 1 : nx;  // wide rows: at least one token row (then one CTA per SM)
   a.nx = nx > kMaxTok ? kMaxTok : nx;
-  size_t off = size_t(warps_of<FMT>()) * a.warp_bytes;
+  size_t off = size_t(warps) * a.warp_bytes;
   a.off_x = int(off);
   off += align256(size_t(a.nx) * a.x_stride);
   a.off_xsum = int(off);
@@ -722,26 +730,41 @@ static bool plan(FfnArgs& a) {
   return off <= 220 * 1024;
 }
 
-template <int FMT, int MODE>
-static cudaError_t launch_one(FfnArgs a, int slots, cudaStream_t st) {
-  if (!plan<FMT>(a)) return cudaErrorInvalidValue;
+template <int FMT, int MODE, int WARPS>
+static cudaError_t launch_plan(const FfnArgs& a, int slots, cudaStream_t st) {
   const size_t smem = size_t(a.off_bits) + 256;
   // raise the kernel's dynamic shared-memory limit once per device (kept out of later
   // calls, which may be inside a graph capture)
-  static bool raised[128] = {};
+  static std::atomic<bool> raised[128] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-  if (!raised[dev]) {
+  if (!raised[dev].load(std::memory_order_relaxed)) {
     cudaError_t err =
-        cudaFuncSetAttribute(k_ffn_gemv<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+        cudaFuncSetAttribute(k_ffn_gemv<FMT, MODE, WARPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
     if (err != cudaSuccess) return err;
-    raised[dev] = true;
+    raised[dev].store(true, std::memory_order_relaxed);
   }
   const int TPE = (MODE == kGateUp) ? a.I / 8 : a.N / kRows;
-  constexpr int W = warps_of<FMT>();
-  k_ffn_gemv<FMT, MODE><<<dim3(unsigned((TPE + W - 1) / W), unsigned(slots)), 32 * W, smem, st>>>(a);
+  k_ffn_gemv<FMT, MODE, WARPS><<<dim3(unsigned((TPE + WARPS - 1) / WARPS), unsigned(slots)), 32 * WARPS, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+// need: tokens an expert may bring (at most T).  Four small CTAs per SM stage up to 16
+// token rows each; when wide rows (large K) leave room for fewer than min(need, 4), an
+// expert's weights would stream once per staged token, so W4 / NVFP4 switch to one CTA of
+// 16 warps per SM, whose single activation stage holds several rows for all 16 warps.
+template <int FMT, int MODE>
+static cudaError_t launch_one(FfnArgs a, int slots, int need, cudaStream_t st) {
+  if (!plan<FMT>(a)) return cudaErrorInvalidValue;
+  if constexpr (FMT != MOE_FMT_BITPLANE8) {
+    if (a.nx < (need < 4 ? need : 4)) {
+      FfnArgs b = a;
+      if (plan<FMT>(b, kWarpsWide, kSmemTargetWide) && b.nx > a.nx)
+        return launch_plan<FMT, MODE, kWarpsWide>(b, slots, st);
+    }
+  }
+  return launch_plan<FMT, MODE, warps_of<FMT>()>(a, slots, st);
 }
 
 template <int FMT>
@@ -757,6 +780,7 @@ static cudaError_t launch_fmt(const uint16_t* x, const moe_routing_t& r, const m
   a.offsets = r.expert_offsets;
   a.sorted_pair = r.sorted_pair;
   a.bits = bits;
+  a.max_rows = INT_MAX;
   // gate/up
   a.act = x;
   a.K = H;
@@ -766,7 +790,7 @@ static cudaError_t launch_fmt(const uint16_t* x, const moe_routing_t& r, const m
   a.gscale = ex.w13_gscale;
   a.out = hbuf;
   a.out_ld = I;
-  cudaError_t err = launch_one<FMT, kGateUp>(a, slots, st);
+  cudaError_t err = launch_one<FMT, kGateUp>(a, slots, T, st);
   if (err != cudaSuccess) return err;
   // down
   a.act = hbuf;
@@ -777,7 +801,53 @@ static cudaError_t launch_fmt(const uint16_t* x, const moe_routing_t& r, const m
   a.gscale = ex.w2_gscale;
   a.out = y_rows;
   a.out_ld = H;
-  return launch_one<FMT, kDown>(a, slots, st);
+  return launch_one<FMT, kDown>(a, slots, T, st);
+}
+
+// One pass (gate/up or down) of the weight-streaming path over the experts with at most
+// max_rows routed rows: the small experts of a batch that otherwise takes the GEMM.  h rows
+// of those experts are written and read in this path's own format (disjoint from the GEMM's).
+template <int FMT>
+static cudaError_t launch_small_fmt(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
+                                    int H, int I, int E, int k, void* hbuf, uint16_t* y_rows, bool down,
+                                    int max_rows, cudaStream_t st) {
+  const int P = T * k;
+  FfnArgs a{};
+  a.k = k;
+  a.I = I;
+  a.expert_list = r.expert_list;
+  a.offsets = r.expert_offsets;
+  a.sorted_pair = r.sorted_pair;
+  a.max_rows = max_rows;
+  if (!down) {
+    a.act = x;
+    a.K = H;
+    a.N = 2 * I;
+    a.w = ex.w13;
+    a.s = ex.w13_scale;
+    a.gscale = ex.w13_gscale;
+    a.out = hbuf;
+    a.out_ld = I;
+    return launch_one<FMT, kGateUp>(a, P < E ? P : E, T < max_rows ? T : max_rows, st);
+  }
+  a.act = hbuf;
+  a.K = I;
+  a.N = H;
+  a.w = ex.w2;
+  a.s = ex.w2_scale;
+  a.gscale = ex.w2_gscale;
+  a.out = y_rows;
+  a.out_ld = H;
+  return launch_one<FMT, kDown>(a, P < E ? P : E, T < max_rows ? T : max_rows, st);
+}
+
+cudaError_t launch_gemv_small(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H, int I,
+                              int E, int k, void* hbuf, uint16_t* y_rows, bool down, int max_rows, cudaStream_t st) {
+  if (ex.fmt == MOE_FMT_W4G128)
+    return launch_small_fmt<MOE_FMT_W4G128>(x, r, ex, T, H, I, E, k, hbuf, y_rows, down, max_rows, st);
+  if (ex.fmt == MOE_FMT_NVFP4)
+    return launch_small_fmt<MOE_FMT_NVFP4>(x, r, ex, T, H, I, E, k, hbuf, y_rows, down, max_rows, st);
+  return cudaErrorInvalidValue;
 }
 
 bool ffn_shape_supported(int64_t H, int64_t I, moe_format_t fmt) {

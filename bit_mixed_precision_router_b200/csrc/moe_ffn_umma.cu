@@ -87,6 +87,10 @@ static_assert(kSmemBytes > 114 * 1024 && kSmemBytes <= 227 * 1024, "shared-memor
 static_assert(kACol0 + kAStages * kACols <= kTmemCols, "tensor-memory plan");
 
 constexpr int kGateUp = 0, kDown = 1;
+// Experts with at most this many routed rows stream through the GEMV even in a GEMM batch:
+// a GEMM tile costs its K/16 MMAs whatever its row count, a GEMV pass reads the weights once
+// for up to 16 tokens.
+constexpr int kSmallRows = 16;
 
 struct UmmaArgs {
   int K, I, E, k;
@@ -99,13 +103,8 @@ struct UmmaArgs {
   const float* gs;           // NVFP4: per-expert fp32 scale of this matrix [E]
   uint16_t* out;             // gate/up: h [P][I] (fp16 h/16 for W4, h/256 for NVFP4); down: y [P][H] bf16
   int out_ld;
+  int min_rows;              // experts with fewer routed rows are left to the weight-streaming GEMV
   unsigned* err;
-  // NVFP4 activations (W4A4): the B operand holds the exact values e2m1 * e4m3 of the
-  // quantised activations, whose tensor's amax is *act_amax (scale amax / 2688); gate/up
-  // then writes h as fp32 to out_f32 and its amax to *out_amax (the next quantisation)
-  const float* act_amax;
-  float* out_f32;
-  float* out_amax;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -287,7 +286,12 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     const int per = (E + 31) / 32;
     const int b = min(E, lane * per), en = min(E, b + per);
     int sum = 0;
-    for (int e = b; e < en; ++e) sum += (offs[e + 1] - offs[e] + kTN - 1) / kTN;
+    // row tiles of expert e (none for an expert below min_rows: the GEMV takes it)
+    auto tiles = [&](int e) {
+      const int n = offs[e + 1] - offs[e];
+      return n < a.min_rows ? 0 : (n + kTN - 1) / kTN;
+    };
+    for (int e = b; e < en; ++e) sum += tiles(e);
     int inc = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -297,7 +301,7 @@ __global__ void __launch_bounds__(kThreadsU, 1)
     int run = inc - sum;
     for (int e = b; e < en; ++e) {
       pre[e] = run;
-      run += (offs[e + 1] - offs[e] + kTN - 1) / kTN;
+      run += tiles(e);
     }
     if (lane == 31) pre[E] = inc;
   } else if (tid == 64) {
@@ -517,11 +521,8 @@ __global__ void __launch_bounds__(kThreadsU, 1)
       if (!warp_wait(&accFull[ab], (it >> 1) & 1, a.err)) break;
       tc_fence_after();
       // the accumulator holds sum w' * x * act_scale (NVFP4: w' = e2m1 * e4m3, the
-      // per-tensor scale still to apply; W4A4: sum w' * a' with a' = e2m1 * e4m3 of the
-      // activations, both per-tensor scales still to apply)
-      float post = (FMT == MOE_FMT_NVFP4) ? 256.f * a.gs[tl.e] : 16.f;
-      if (FMT == MOE_FMT_NVFP4 && a.act_amax) post = a.gs[tl.e] * __fdiv_rn(*a.act_amax, 2688.0f);
-      float amax = 0.f;
+      // per-tensor scale still to apply)
+      const float post = (FMT == MOE_FMT_NVFP4) ? 256.f * a.gs[tl.e] : 16.f;
       for (int c0 = 0; c0 < tl.nrows; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + uint32_t(ab * kTN + c0), v);
@@ -541,20 +542,10 @@ __global__ void __launch_bounds__(kThreadsU, 1)
             const float up = __shfl_xor_sync(0xffffffffu, mine, 16);
             if (lane < 16 && c < nc) {
               const float hv = silu(mine) * up;
-              if (a.out_f32) {
-                a.out_f32[size_t(tl.r0 + c0 + c) * a.out_ld + tl.wt * 64 + quarter * 16 + lane] = hv;
-                amax = fmaxf(amax, fabsf(hv));
-              } else {
-                o[size_t(c) * a.out_ld] = __half_as_ushort(__float2half_rn(hv * act_scale<FMT>()));
-              }
+              o[size_t(c) * a.out_ld] = __half_as_ushort(__float2half_rn(hv * act_scale<FMT>()));
             }
           }
         }
-      }
-      if (MODE == kGateUp && a.out_f32) {
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (lane == 0) atomicMax(reinterpret_cast<unsigned*>(a.out_amax), __float_as_uint(amax));
       }
       tc_fence_before();
       __syncwarp();
@@ -605,31 +596,6 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x
       }
     }
   }
-}
-
-// B operand of the W4A4 GEMMs: row r of dst = the exact fp16 values e2m1 * e4m3 of the
-// NVFP4 activation row src(r) (gate/up: the token of routed row r; down: r itself).  One
-// thread per block of 16 elements (8 code bytes, one E4M3 scale -> 32 bytes of fp16).
-__global__ void __launch_bounds__(256) k_dequant_rows_nvfp4(const uint8_t* __restrict__ codes,
-                                                            const uint8_t* __restrict__ sb,
-                                                            const int32_t* __restrict__ sorted_pair, int k,
-                                                            int64_t nblocks, int C16, uint4* __restrict__ dst) {
-  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-  if (i >= nblocks) return;
-  const int64_t r = i / C16;
-  const int b = int(i - r * C16);
-  const int64_t src = sorted_pair ? int64_t(__ldg(sorted_pair + r) / k) : r;
-  const int64_t blk = src * C16 + b;
-  const uint2 cw = *reinterpret_cast<const uint2*>(codes + blk * 8);
-  const uint32_t s2 = e4m3_to_h2(sb[blk]);
-  uint32_t o[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    o[j] = hmul2(e2m1x2_to_h2((cw.x >> (8 * j)) & 0xFFu), s2);
-    o[4 + j] = hmul2(e2m1x2_to_h2((cw.y >> (8 * j)) & 0xFFu), s2);
-  }
-  dst[i * 2] = make_uint4(o[0], o[1], o[2], o[3]);
-  dst[i * 2 + 1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // ---------------------------------------------------------------- host side
@@ -692,6 +658,380 @@ cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- W4A4 on the FP4 tensor cores
+// tcgen05.mma kind::mxf4nvf4 with block16 scales: A = 128 weight rows of E2M1 codes, B = 128
+// routed rows of E2M1 codes, both from shared memory (K-major, 128-byte swizzle; 256 codes
+// = 128 bytes per row per stage), their E4M3 block scales in tensor memory.  Per 64-element
+// K block (one MMA) a scale block of 512 bytes holds, for tile row m = m0 + 32 m1 and its
+// four 16-element sub-blocks kk, the byte 16 m0 + 4 m1 + kk; tcgen05.cp (32x128b, warpx4)
+// puts it into four tensor-memory columns of every lane quarter: lane 32 r + m0, column m1,
+// byte kk.  The weight scales are laid out that way once per call from the row-major
+// scales (k_sf_tiles); the activation scales by their quantiser's row scatter.
+constexpr int kF4TM = 128, kF4TN = 128;
+constexpr int kF4Stages = 6;                        // K stages of 256 elements (128 bytes per row)
+constexpr int kF4ABytes = kF4TM * 128, kF4BBytes = kF4TN * 128, kF4SfBytes = 4 * 512;
+constexpr int kF4StageBytes = kF4ABytes + kF4BBytes + 2 * kF4SfBytes;  // 36 KiB
+constexpr int kF4OffPre = kF4Stages * kF4StageBytes;
+constexpr int kF4OffOffs = kF4OffPre + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
+constexpr int kF4OffBar = kF4OffOffs + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
+constexpr int kF4NumBars = 2 * kF4Stages + 4;
+constexpr int kF4OffTmemSlot = kF4OffBar + kF4NumBars * 8;
+constexpr int kF4SmemBytes = kF4OffTmemSlot + 16 + 1024;
+constexpr int kF4Threads = 256;                     // producer, MMA, 2 idle, 4 epilogue warps
+// tensor-memory columns: accumulators at 0 and 128, the scales of stage s at 256 + 32 s (A)
+// and 272 + 32 s (B), 4 columns per 64-element K block
+constexpr uint32_t kF4SfaCol = 2 * kF4TN, kF4SfbCol = 2 * kF4TN + 16, kF4SfStageCols = 32;
+static_assert(kF4SfaCol + kF4Stages * kF4SfStageCols <= 512, "tensor-memory plan");
+static_assert(kF4SmemBytes <= 227 * 1024, "shared-memory plan");
+static_assert(kF4StageBytes % 1024 == 0, "stage alignment for the 128-byte swizzle");
+
+struct F4Args {
+  int K, I, E, wtiles, n_rows;
+  const int32_t* offsets;
+  const uint8_t* sfa;       // weight scales, tiled: [E][wtiles][K/64][512]
+  const uint8_t* sfb;       // activation scales, tiled: [row tiles][K/64][512]
+  const float* gs;          // per-expert weight scale of this matrix [E]
+  const float* act_amax;    // amax of the activation tensor (scale amax / 2688)
+  uint16_t* out;            // down: y bf16 [P][H]
+  int out_ld;
+  float* out_f32;           // gate/up: h fp32 [P][I]
+  float* out_amax;          // gate/up: amax of h
+  unsigned* err;
+};
+
+// Shared-memory descriptor of a 512-byte scale block for tcgen05.cp: K-major, no swizzle,
+// 16-byte rows, 8-row core matrices 128 bytes apart.
+MOE_DEVICE uint64_t sf_desc(uint32_t saddr) {
+  uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t(1) << 16;          // leading byte offset (one core matrix along K)
+  d |= uint64_t(128 >> 4) << 32;   // stride byte offset: next 8 rows
+  d |= uint64_t(1) << 46;          // descriptor version
+  return d;                        // layout type 0: no swizzle
+}
+MOE_DEVICE void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T with E4M3 block-16 scales from tensor memory; M = 128, K = 64.
+MOE_DEVICE void tc_mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t sfa,
+                           uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Instruction descriptor (block-scaled): A and B E2M1 (format 1), K-major, E4M3 scales,
+// N = 128, M = 128, scale ids 0.
+constexpr uint32_t kF4Idesc = (1u << 7) | (1u << 10) | (uint32_t(kF4TN >> 3) << 17) | (uint32_t(kF4TM >> 4) << 24);
+
+MOE_DEVICE Tile tile_of_n(int item, const int* pre, int E, int wtiles, const int* offsets, int tn, int* rtile) {
+  const int t = item / wtiles;
+  Tile tl;
+  tl.wt = item - t * wtiles;
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pre[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  tl.e = lo;
+  const int beg = offsets[lo], end = offsets[lo + 1];
+  tl.r0 = beg + (t - pre[lo]) * tn;
+  tl.nrows = min(tn, end - tl.r0);
+  *rtile = t;
+  return tl;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kF4Threads, 1)
+    k_ffn_fp4(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w, F4Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
+  int* pre = reinterpret_cast<int*>(smem + kF4OffPre);
+  int* offs = reinterpret_cast<int*>(smem + kF4OffOffs);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF4OffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kF4Stages;
+  uint64_t* accFull = empty + kF4Stages;
+  uint64_t* accEmpty = accFull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kF4OffTmemSlot);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = a.E;
+
+  for (int i = tid; i <= E; i += blockDim.x) offs[i] = a.offsets[i];
+  __syncthreads();
+  if (warp == 0) {  // row tiles of kF4TN per expert, and their prefix
+    const int per = (E + 31) / 32;
+    const int b = min(E, lane * per), en = min(E, b + per);
+    int sum = 0;
+    for (int e = b; e < en; ++e) sum += (offs[e + 1] - offs[e] + kF4TN - 1) / kF4TN;
+    int inc = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += v;
+    }
+    int run = inc - sum;
+    for (int e = b; e < en; ++e) {
+      pre[e] = run;
+      run += (offs[e + 1] - offs[e] + kF4TN - 1) / kF4TN;
+    }
+    if (lane == 31) pre[E] = inc;
+  } else if (tid == 64) {
+    for (int i = 0; i < kF4Stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accFull[i], 1);
+      mbar_init(&accEmpty[i], 4);
+    }
+    fence_mbar_init();
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = pre[E] * a.wtiles;
+  const int KB64 = a.K / 64, KS = (KB64 + 3) / 4;  // the last stage may hold 2 of its 4 K blocks
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    int n = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      int rt = 0;
+      const Tile tl = tile_of_n(item, pre, E, a.wtiles, offs, kF4TN, &rt);
+      for (int ks = 0; ks < KS; ++ks, ++n) {
+        const int s = n % kF4Stages;
+        if (!warp_wait(&empty[s], ((n / kF4Stages) & 1) ^ 1, a.err)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t st = sbase + s * kF4StageBytes;
+          const uint32_t sf_bytes = uint32_t(min(4, KB64 - 4 * ks)) * 512u;
+          mbar_arrive_expect_tx(&full[s], uint32_t(kF4ABytes + kF4BBytes) + 2 * sf_bytes);
+          if (MODE == kGateUp) {  // rows 32q..32q+15: gate rows 16q.., 32q+16..: the matching up rows
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int g0 = tl.e * a.n_rows + tl.wt * 64 + 16 * q;
+              tma_load_2d(st + (32 * q) * 128, &tm_w, ks * 128, g0, &full[s]);
+              tma_load_2d(st + (32 * q + 16) * 128, &tm_w, ks * 128, g0 + a.I, &full[s]);
+            }
+          } else {
+            tma_load_2d(st, &tm_w, ks * 128, tl.e * a.n_rows + tl.wt * kF4TM, &full[s]);
+          }
+          tma_load_2d(st + kF4ABytes, &tm_b, ks * 128, tl.r0, &full[s]);
+          bulk_g2s(smem + s * kF4StageBytes + kF4ABytes + kF4BBytes,
+                   a.sfa + (size_t(tl.e * a.wtiles + tl.wt) * KB64 + 4 * ks) * 512, sf_bytes, &full[s]);
+          bulk_g2s(smem + s * kF4StageBytes + kF4ABytes + kF4BBytes + kF4SfBytes,
+                   a.sfb + (size_t(rt) * KB64 + 4 * ks) * 512, sf_bytes, &full[s]);
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      int n = 0, it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
+        const int ab = it & 1;
+        if (!mbar_wait(&accEmpty[ab], ((it >> 1) & 1) ^ 1, a.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + uint32_t(ab * kF4TN);
+        for (int ks = 0; ks < KS; ++ks, ++n) {
+          const int s = n % kF4Stages;
+          if (!mbar_wait(&full[s], (n / kF4Stages) & 1, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + s * kF4StageBytes;
+          const uint32_t sfa = tmem + kF4SfaCol + kF4SfStageCols * s, sfb = tmem + kF4SfbCol + kF4SfStageCols * s;
+          const int nkb = min(4, KB64 - 4 * ks);
+          const uint64_t adesc = sw128_desc(st), bdesc = sw128_desc(st + kF4ABytes);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            if (kb < nkb) {
+              tc_cp_sf(sfa + 4 * kb, sf_desc(st + kF4ABytes + kF4BBytes + 512 * kb));
+              tc_cp_sf(sfb + 4 * kb, sf_desc(st + kF4ABytes + kF4BBytes + kF4SfBytes + 512 * kb));
+            }
+          }
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)  // 32 bytes (64 codes) per MMA inside the 128-byte row
+            if (kb < nkb)
+              tc_mma_fp4(d_tmem, adesc + uint64_t(2 * kb), bdesc + uint64_t(2 * kb), kF4Idesc, sfa + 4 * kb,
+                         sfb + 4 * kb, (ks | kb) != 0);
+          tc_commit(&empty[s]);
+        }
+        if (ok) tc_commit(&accFull[ab]);
+      }
+      if (it > 0 && ok) mbar_wait(&accFull[(it - 1) & 1], ((it - 1) >> 1) & 1, a.err);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------ epilogue
+    const int quarter = warp - 4;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+      int rt = 0;
+      const Tile tl = tile_of_n(item, pre, E, a.wtiles, offs, kF4TN, &rt);
+      const int ab = it & 1;
+      if (!warp_wait(&accFull[ab], (it >> 1) & 1, a.err)) break;
+      tc_fence_after();
+      const float post = a.gs[tl.e] * __fdiv_rn(*a.act_amax, 2688.0f);
+      float amax = 0.f;
+      for (int c0 = 0; c0 < tl.nrows; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + uint32_t(ab * kF4TN + c0), v);
+        tc_wait_ld();
+        const int nc = min(32, tl.nrows - c0);
+        if (MODE == kDown) {
+          uint16_t* o = a.out + size_t(tl.r0 + c0) * a.out_ld + tl.wt * kF4TM + quarter * 32 + lane;
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c < nc) o[size_t(c) * a.out_ld] = float_to_bf16_bits(__uint_as_float(v[c]) * post);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float mine = __uint_as_float(v[c]) * post;
+            const float up = __shfl_xor_sync(0xffffffffu, mine, 16);
+            if (lane < 16 && c < nc) {
+              const float hv = silu(mine) * up;
+              a.out_f32[size_t(tl.r0 + c0 + c) * a.out_ld + tl.wt * 64 + quarter * 16 + lane] = hv;
+              amax = fmaxf(amax, fabsf(hv));
+            }
+          }
+        }
+      }
+      if (MODE == kGateUp) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) atomicMax(reinterpret_cast<unsigned*>(a.out_amax), __float_as_uint(amax));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accEmpty[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Weight scales, row-major E4M3 [E][N][K/16] -> tiled [E][wtiles][K/64][512]: tile wt, K block
+// kb, tile row m = m0 + 32 m1 (gate/up: m1 = q, m0 < 16 the gate row 64 wt + 16 q + m0, else
+// the up row I + 64 wt + 16 q + m0 - 16; down: row 128 wt + m), byte 16 m0 + 4 m1 + kk.
+// One thread per (E, wtile, kb, m0): 16 bytes.
+__global__ void k_sf_tiles_w(const uint8_t* __restrict__ sb, int E, int N, int K, int I, int gate_up,
+                             uint8_t* __restrict__ out) {
+  const int KB = K / 64, wtiles = gate_up ? I / 64 : N / 128;
+  const int64_t total = int64_t(E) * wtiles * KB * 32;
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= total) return;
+  const int m0 = int(i % 32);
+  int64_t r = i / 32;
+  const int kb = int(r % KB);
+  r /= KB;
+  const int wt = int(r % wtiles);
+  const int e = int(r / wtiles);
+  uint32_t w[4];
+#pragma unroll
+  for (int m1 = 0; m1 < 4; ++m1) {
+    int row;
+    if (gate_up) row = (m0 < 16) ? 64 * wt + 16 * m1 + m0 : I + 64 * wt + 16 * m1 + (m0 - 16);
+    else row = 128 * wt + 32 * m1 + m0;
+    w[m1] = *reinterpret_cast<const uint32_t*>(sb + (size_t(e) * N + row) * (K / 16) + 4 * kb);
+  }
+  *reinterpret_cast<uint4*>(out + ((size_t(e) * wtiles + wt) * KB + kb) * 512 + 16 * m0) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Row tiles of kF4TN routed rows per expert: pre[e] for e <= E (one CTA).
+__global__ void __launch_bounds__(1024) k_row_tile_prefix(const int32_t* __restrict__ offsets, int E,
+                                                          int32_t* __restrict__ pre) {
+  __shared__ int part[1024];
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int b = min(E, int(threadIdx.x) * per), en = min(E, b + per);
+  int sum = 0;
+  for (int e = b; e < en; ++e) sum += (offsets[e + 1] - offsets[e] + kF4TN - 1) / kF4TN;
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  for (int d = 1; d < int(blockDim.x); d <<= 1) {
+    const int v = int(threadIdx.x) >= d ? part[threadIdx.x - d] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int run = part[threadIdx.x] - sum;
+  for (int e = b; e < en; ++e) {
+    pre[e] = run;
+    run += (offsets[e + 1] - offsets[e] + kF4TN - 1) / kF4TN;
+  }
+  if (threadIdx.x == blockDim.x - 1) pre[E] = part[threadIdx.x];
+}
+
+// B operand rows in routed order and their tiled scales: routed row r of expert e (tile
+// pre[e] + (r - off_e) / 128, tile row n = (r - off_e) % 128) takes the codes of source row
+// src(r) (gate/up: its token; down: r) and scatters its E4M3 scales to byte 16 (n % 32) +
+// 4 (n / 32) + kk of K block kb.  One thread per (row, K block of 64): 32 code bytes, 4 scales.
+__global__ void k_route_fp4_rows(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sb,
+                                 const int32_t* __restrict__ sorted_pair, int k, const int32_t* __restrict__ offsets,
+                                 int E, const int32_t* __restrict__ pre, int P, int K, uint8_t* __restrict__ codes_out,
+                                 uint8_t* __restrict__ sf_out) {
+  const int KB = K / 64;
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= int64_t(P) * KB) return;
+  const int r = int(i / KB), kb = int(i - int64_t(r) * KB);
+  int lo = 0, hi = E;  // expert of row r: largest e with offsets[e] <= r
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offsets[mid] <= r) lo = mid;
+    else hi = mid;
+  }
+  const int nrow = r - offsets[lo];
+  const int tile = pre[lo] + nrow / kF4TN, n = nrow % kF4TN;
+  const int64_t src = sorted_pair ? int64_t(sorted_pair[r] / k) : int64_t(r);
+  if (codes_out) {
+    const uint4* cs = reinterpret_cast<const uint4*>(codes + src * (K / 2) + kb * 32);
+    uint4* cd = reinterpret_cast<uint4*>(codes_out + int64_t(r) * (K / 2) + kb * 32);
+    cd[0] = cs[0];
+    cd[1] = cs[1];
+  }
+  const uint32_t s4 = *reinterpret_cast<const uint32_t*>(sb + src * (K / 16) + 4 * kb);
+  *reinterpret_cast<uint32_t*>(sf_out + (size_t(tile) * KB + kb) * 512 + 16 * (n % 32) + 4 * (n / 32)) = s4;
+}
+
+template <int MODE>
+cudaError_t launch_fp4_one(const CUtensorMap& tb, const CUtensorMap& tw, const F4Args& a, cudaStream_t st) {
+  static std::atomic<bool> raised[128] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (!raised[dev].load(std::memory_order_relaxed)) {
+    const cudaError_t err = cudaFuncSetAttribute(k_ffn_fp4<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kF4SmemBytes);
+    if (err != cudaSuccess) return err;
+    raised[dev].store(true, std::memory_order_relaxed);
+  }
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  k_ffn_fp4<MODE><<<nsm, kF4Threads, kF4SmemBytes, st>>>(tb, tw, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 // At 32 or more rows per expert on average, the tensor-core GEMM (weights
@@ -717,6 +1057,7 @@ static cudaError_t launch_umma_fmt(const uint16_t* x, const moe_routing_t& r, co
   a.I = I;
   a.offsets = r.expert_offsets;
   a.sorted_pair = r.sorted_pair;
+  a.min_rows = kSmallRows + 1;
   a.err = device_error_word();
   if (!a.err) return cudaErrorInvalidDevice;
   const int nsm = sm_count();
@@ -746,6 +1087,8 @@ static cudaError_t launch_umma_fmt(const uint16_t* x, const moe_routing_t& r, co
   a.out_ld = I;
   err = launch_umma_one<FMT, kGateUp>(tb, tw, a, st);
   if (err != cudaSuccess) return err;
+  err = launch_gemv_small(x, r, ex, T, H, I, E, k, hbuf, y_rows, false, kSmallRows, st);
+  if (err != cudaSuccess) return err;
   // down: h rows, two 64-K boxes per stage; weight boxes of 128 rows
   if (!make_map_2d(&tb, act_type, hbuf, uint64_t(I), uint64_t(P), uint64_t(I) * 2, kAtomK, kTN,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -760,7 +1103,9 @@ static cudaError_t launch_umma_fmt(const uint16_t* x, const moe_routing_t& r, co
   a.gs = ex.w2_gscale;
   a.out = y_rows;
   a.out_ld = H;
-  return launch_umma_one<FMT, kDown>(tb, tw, a, st);
+  err = launch_umma_one<FMT, kDown>(tb, tw, a, st);
+  if (err != cudaSuccess) return err;
+  return launch_gemv_small(x, r, ex, T, H, I, E, k, hbuf, y_rows, true, kSmallRows, st);
 }
 
 cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
@@ -772,13 +1117,30 @@ cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, c
 }
 
 // ---------------------------------------------------------------- W4A4 (NVFP4 activations)
-// Workspace: two amax words, x codes [T][H/2] and scales [T][H/16], the routed B rows
-// fp16 [P][H], h fp32 [P][I], h codes [P][I/2] and scales [P][I/16], h B rows fp16 [P][I].
+// Weight scales in the tensor-memory copy order, written once per set of experts: w13's
+// [E][I/64][H/64][512] (gate/up tiles interleave 16 gate and 16 up rows), then w2's
+// [E][H/128][I/64][512].
+size_t w4a4_scale_tiles_bytes(int64_t H, int64_t I, int64_t E) {
+  return align256u(size_t(E * 2 * I * H / 16)) + align256u(size_t(E * H * I / 16));
+}
+
+cudaError_t launch_w4a4_prepare(const moe_experts_t& ex, int H, int I, int E, uint8_t* tiles, cudaStream_t st) {
+  const int64_t n13 = int64_t(E) * (I / 64) * (H / 64) * 32, n2 = int64_t(E) * (H / 128) * (I / 64) * 32;
+  k_sf_tiles_w<<<unsigned((n13 + 255) / 256), 256, 0, st>>>(static_cast<const uint8_t*>(ex.w13_scale), E, 2 * I, H, I,
+                                                            1, tiles);
+  k_sf_tiles_w<<<unsigned((n2 + 255) / 256), 256, 0, st>>>(static_cast<const uint8_t*>(ex.w2_scale), E, H, I, I, 0,
+                                                           tiles + align256u(size_t(int64_t(E) * 2 * I * H / 16)));
+  return cudaGetLastError();
+}
+
+// Workspace: two amax words, the row-tile prefix, x codes [T][H/2] and scales [T][H/16], the
+// routed x codes [P][H/2] and their tiled scales, h fp32 [P][I], h codes [P][I/2] and scales
+// [P][I/16], and h's tiled scales.
 struct W4a4Plan {
-  size_t amax, xc, xsb, bx, hf, hc, hsb, bh, total;
+  size_t amax, pre, xc, xsb, bxc, sfbx, hf, hc, hsb, sfbh, total;
 };
-static W4a4Plan w4a4_plan(int64_t T, int64_t H, int64_t I, int64_t k) {
-  const int64_t P = T * k;
+static W4a4Plan w4a4_plan(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
+  const int64_t P = T * k, tiles = P / kF4TN + E;  // row tiles: sum over experts of ceil(n_e / 128)
   W4a4Plan p{};
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -787,87 +1149,95 @@ static W4a4Plan w4a4_plan(int64_t T, int64_t H, int64_t I, int64_t k) {
     return at;
   };
   p.amax = take(256);
+  p.pre = take(size_t(E + 1) * 4);
   p.xc = take(size_t(T * H / 2));
   p.xsb = take(size_t(T * H / 16));
-  p.bx = take(size_t(P * H * 2));
+  p.bxc = take(size_t(P * H / 2));
+  p.sfbx = take(size_t(tiles * (H / 64) * 512));
   p.hf = take(size_t(P * I * 4));
   p.hc = take(size_t(P * I / 2));
   p.hsb = take(size_t(P * I / 16));
-  p.bh = take(size_t(P * I * 2));
+  p.sfbh = take(size_t(tiles * (I / 64) * 512));
   p.total = o;
   return p;
 }
 
-size_t w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k) { return w4a4_plan(T, H, I, k).total; }
+size_t w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
+  return w4a4_plan(T, H, I, E, k).total;
+}
 
-cudaError_t launch_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H,
-                                    int I, int E, int k, uint16_t* y_rows, void* ws, cudaStream_t st) {
+cudaError_t launch_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
+                                    const uint8_t* tiles, int T, int H, int I, int E, int k, uint16_t* y_rows,
+                                    void* ws, cudaStream_t st) {
   const int P = T * k;
-  const W4a4Plan pl = w4a4_plan(T, H, I, k);
+  const W4a4Plan pl = w4a4_plan(T, H, I, E, k);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* amax_x = reinterpret_cast<float*>(base + pl.amax);
   float* amax_h = amax_x + 1;
-  const int nsm = sm_count();
-  if (nsm <= 0) return cudaErrorInvalidDevice;
-  // x -> NVFP4 (one tensor), then its exact values in routed-row order
-  cudaError_t err = launch_act_nvfp4<uint16_t>(x, int64_t(T) * H, base + pl.xc, base + pl.xsb, amax_x, st);
+  int32_t* pre = reinterpret_cast<int32_t*>(base + pl.pre);
+  cudaError_t err;
+  k_row_tile_prefix<<<1, 1024, 0, st>>>(r.expert_offsets, E, pre);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  // x -> NVFP4 (one tensor), then its codes in routed-row order and its scales tiled
+  err = launch_act_nvfp4<uint16_t>(x, int64_t(T) * H, base + pl.xc, base + pl.xsb, amax_x, st);
   if (err != cudaSuccess) return err;
-  int64_t nb = int64_t(P) * (H / 16);
-  k_dequant_rows_nvfp4<<<unsigned((nb + 255) / 256), 256, 0, st>>>(base + pl.xc, base + pl.xsb, r.sorted_pair, k, nb,
-                                                                   H / 16, reinterpret_cast<uint4*>(base + pl.bx));
+  int64_t nb = int64_t(P) * (H / 64);
+  k_route_fp4_rows<<<unsigned((nb + 255) / 256), 256, 0, st>>>(base + pl.xc, base + pl.xsb, r.sorted_pair, k,
+                                                               r.expert_offsets, E, pre, P, H, base + pl.bxc,
+                                                               base + pl.sfbx);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if ((err = cudaMemsetAsync(amax_h, 0, sizeof(float), st)) != cudaSuccess) return err;
-  UmmaArgs a{};
+  F4Args a{};
   a.E = E;
-  a.k = k;
   a.I = I;
   a.offsets = r.expert_offsets;
-  a.sorted_pair = r.sorted_pair;
   a.err = device_error_word();
   if (!a.err) return cudaErrorInvalidDevice;
   CUtensorMap tb, tw;
-  // gate/up: B = the routed rows of x's exact values, h written as fp32 with its amax
-  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + pl.bx, uint64_t(H), uint64_t(P), uint64_t(H) * 2,
-                   kAtomK, kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // gate/up: weight boxes of 16 rows (gate and up interleaved per 16), B boxes of 128 rows
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, base + pl.bxc, uint64_t(H) / 2, uint64_t(P), uint64_t(H) / 2,
+                   128, kF4TN, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w13, uint64_t(H) / 2, uint64_t(E) * 2 * I,
-                   uint64_t(H) / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+                   uint64_t(H) / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   a.K = H;
   a.n_rows = 2 * I;
   a.wtiles = I / 64;
-  a.bs = static_cast<const uint8_t*>(ex.w13_scale);
+  a.sfa = tiles;
+  a.sfb = base + pl.sfbx;
   a.gs = ex.w13_gscale;
+  a.act_amax = amax_x;
   a.out = nullptr;
   a.out_ld = I;
-  a.act_amax = amax_x;
   a.out_f32 = reinterpret_cast<float*>(base + pl.hf);
   a.out_amax = amax_h;
-  err = launch_umma_one<MOE_FMT_NVFP4, kGateUp>(tb, tw, a, st);
+  err = launch_fp4_one<kGateUp>(tb, tw, a, st);
   if (err != cudaSuccess) return err;
-  // h (fp32, its amax already taken by the epilogue) -> NVFP4, exact values as the down B
-  nb = int64_t(P) * (I / 16);
+  // h (fp32, its amax taken by the epilogue) -> NVFP4 codes in routed order; scales tiled
   err = launch_act_nvfp4_codes<float>(reinterpret_cast<const float*>(base + pl.hf), int64_t(P) * I, base + pl.hc,
                                       base + pl.hsb, amax_h, st);
   if (err != cudaSuccess) return err;
-  k_dequant_rows_nvfp4<<<unsigned((nb + 255) / 256), 256, 0, st>>>(base + pl.hc, base + pl.hsb, nullptr, 1, nb,
-                                                                   I / 16, reinterpret_cast<uint4*>(base + pl.bh));
+  nb = int64_t(P) * (I / 64);
+  k_route_fp4_rows<<<unsigned((nb + 255) / 256), 256, 0, st>>>(nullptr, base + pl.hsb, nullptr, 1, r.expert_offsets,
+                                                               E, pre, P, I, nullptr, base + pl.sfbh);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base + pl.bh, uint64_t(I), uint64_t(P), uint64_t(I) * 2,
-                   kAtomK, kTN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 64,
-                   kTM, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, base + pl.hc, uint64_t(I) / 2, uint64_t(P), uint64_t(I) / 2,
+                   128, kF4TN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, ex.w2, uint64_t(I) / 2, uint64_t(E) * H, uint64_t(I) / 2, 128,
+                   kF4TM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   a.K = I;
   a.n_rows = H;
-  a.wtiles = H / kTM;
-  a.bs = static_cast<const uint8_t*>(ex.w2_scale);
+  a.wtiles = H / kF4TM;
+  a.sfa = tiles + align256u(size_t(int64_t(E) * 2 * I * H / 16));
+  a.sfb = base + pl.sfbh;
   a.gs = ex.w2_gscale;
+  a.act_amax = amax_h;
   a.out = y_rows;
   a.out_ld = H;
-  a.act_amax = amax_h;
   a.out_f32 = nullptr;
   a.out_amax = nullptr;
-  return launch_umma_one<MOE_FMT_NVFP4, kDown>(tb, tw, a, st);
+  return launch_fp4_one<kDown>(tb, tw, a, st);
 }
 
 }  // namespace moe

@@ -42,6 +42,9 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, const moe_routing_t& r, const 
 bool use_umma_path(int64_t T, int64_t E, int64_t k, moe_format_t fmt);
 size_t umma_h_bytes(int64_t T, int64_t I, int64_t k);
 size_t umma_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
+// the weight-streaming pass over the experts with at most max_rows routed rows (GEMM batches)
+cudaError_t launch_gemv_small(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H, int I,
+                              int E, int k, void* hbuf, uint16_t* y_rows, bool down, int max_rows, cudaStream_t st);
 cudaError_t launch_grouped_ffn_umma(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T,
                                     int H, int I, int E, int k, uint16_t* y_rows, void* hbuf, cudaStream_t st);
 
@@ -56,10 +59,14 @@ cudaError_t launch_act_nvfp4_codes(const In* a, int64_t n, uint8_t* codes, uint8
 cudaError_t launch_quantize_nvfp4_f32(const float* a, int64_t n, uint8_t* codes, uint8_t* block_scales,
                                       float* gscale, cudaStream_t st);
 
-// W4A4 prefill (moe_ffn_umma.cu): NVFP4 weights and NVFP4 activations on the tcgen05 GEMM.
-size_t w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t k);
-cudaError_t launch_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex, int T, int H,
-                                    int I, int E, int k, uint16_t* y_rows, void* ws, cudaStream_t st);
+// W4A4 prefill (moe_ffn_umma.cu): NVFP4 weights and NVFP4 activations on the block-scaled
+// FP4 tensor cores; the weight scales first laid out once in the tensor-memory copy order.
+size_t w4a4_scale_tiles_bytes(int64_t H, int64_t I, int64_t E);
+cudaError_t launch_w4a4_prepare(const moe_experts_t& ex, int H, int I, int E, uint8_t* tiles, cudaStream_t st);
+size_t w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k);
+cudaError_t launch_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t& r, const moe_experts_t& ex,
+                                    const uint8_t* tiles, int T, int H, int I, int E, int k, uint16_t* y_rows,
+                                    void* ws, cudaStream_t st);
 
 // Budgeted per-expert bit allocation (moe_alloc.cu).
 cudaError_t launch_bitplane_distortion(const uint32_t* planes, const uint16_t* scales, int E, int N, int K,

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 /* Size limits enforced by validation. */
 #define MOE_MAX_EXPERTS 1024 /* E */
@@ -383,6 +383,22 @@ moe_status_t moe_grouped_ffn(const uint16_t* x, const moe_routing_t* routing,
                              uint16_t* y_rows, void* workspace, size_t workspace_bytes,
                              moe_stream_t stream);
 
+/* Bytes of the weight-scale tiles moe_w4a4_prepare writes for E experts of H, I. */
+size_t moe_w4a4_scale_tiles_bytes(int64_t H, int64_t I, int64_t E);
+
+/* Lays out the E4M3 block scales of NVFP4 experts (as written by moe_quantize_nvfp4) in the
+ * order the block-scaled FP4 tensor cores read them [MoET: NVFP4 for expert GEMMs]: per
+ * 128-row weight tile and 64-element K block, 512 bytes holding the scale of tile row
+ * m = m0 + 32 m1 and sub-block kk (16 elements) at byte 16 m0 + 4 m1 + kk.  Gate/up tiles
+ * are 64 gate and 64 up rows, interleaved by 16 (tile row 32 q + j: gate row 64 t + 16 q + j
+ * for j < 16, else up row I + 64 t + 16 q + j - 16); down tiles are 128 consecutive rows of w2.
+ * Run once per set of experts (the tiles depend on the weights only); the result is read
+ * by every moe_grouped_ffn_w4a4 call on those experts.
+ *   scale_tiles: device, 16-byte aligned, >= moe_w4a4_scale_tiles_bytes(H, I, E) bytes.
+ * Requires H % 256 == 0, I % 128 == 0. */
+moe_status_t moe_w4a4_prepare(const moe_experts_t* experts, int64_t H, int64_t I, int64_t E, void* scale_tiles,
+                              size_t scale_tiles_bytes, moe_stream_t stream);
+
 /* Bytes of device workspace moe_grouped_ffn_w4a4 needs. */
 size_t moe_ffn_w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k);
 
@@ -391,17 +407,20 @@ size_t moe_ffn_w4a4_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, 
  * recipe (E2M1 codes, an E4M3 scale per 16 consecutive elements of a row, one fp32 scale
  * amax/2688 for the tensor); per expert g, u = x' W13'^T, h = silu(g) u kept in fp32; all
  * routed rows of h are quantised the same way, as one tensor, from those fp32 values; y_rows
- * = h' W2'^T (bf16).  Every product is exact: the tensor cores multiply the exact values
- * e2m1 * e4m3 of both operands (fp16, fp32 accumulation) and the two per-tensor scales
- * multiply each sum once.  Always the tcgen05 GEMM (any batch size).
- *   experts: fmt must be MOE_FMT_NVFP4 (as written by moe_quantize_nvfp4); other arguments
- *   and layouts as for moe_grouped_ffn; workspace >= moe_ffn_w4a4_workspace_bytes(...)
- *   (scratch: the quantised x and h, their fp16 values in routed order, h in fp32).
+ * = h' W2'^T (bf16).  The tensor cores take both operands as E2M1 codes with their E4M3
+ * block scales (tcgen05 kind::mxf4nvf4, block16: every product e2m1 * e4m3 * e2m1 * e4m3 is
+ * exact, fp32 accumulation); the two per-tensor scales multiply each sum once.  Always this
+ * GEMM (any batch size): tiles of 128 weight rows x 128 routed rows, K stages of 256.
+ *   experts: fmt must be MOE_FMT_NVFP4; scale_tiles: written by moe_w4a4_prepare for the
+ *   same experts; other arguments and layouts as for moe_grouped_ffn; workspace >=
+ *   moe_ffn_w4a4_workspace_bytes(...) (scratch: the quantised x and h, x's codes in routed
+ *   order, the activation scales in tile order, h in fp32).
+ * Requires H % 256 == 0, I % 128 == 0.
  * Tolerance against the W4A4 definition as for moe_grouped_ffn; an element of h within a
  * rounding of an E2M1 decision boundary may take the other code (fp32 order). */
 moe_status_t moe_grouped_ffn_w4a4(const uint16_t* x, const moe_routing_t* routing, const moe_experts_t* experts,
-                                  int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, uint16_t* y_rows,
-                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
+                                  const void* scale_tiles, int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                                  uint16_t* y_rows, void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* Routing-weighted combine [ExactMoE: the selected experts' outputs weighted by the
  * unchanged routing weights]: out[t] = bf16( sum_{j<k} topk_w[t*k+j] *

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_function(lib):
     for n in sorted(names):
         assert hasattr(lib, n), n
     assert set(moe.exported_symbols()) == names  # the binding covers the whole ABI
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     assert lib.moe_status_string(3) == b"workspace missing or too small"
     assert lib.moe_status_string(99) == b"unknown status"
 
@@ -104,6 +104,39 @@ def test_ffn_and_combine_validation(lib):
     assert c(4, 2048, 0) == INVALID
     assert c(4, 2048, 8, res=A + 8) == MISALIGNED
     assert c(0, 2048, 8) == OK
+
+
+def test_w4a4_validation(lib):
+    r = _routing()
+    ex = ExpertsT(2, A, A, A, A, A, A)
+    H, I, E, k = 2048, 1024, 64, 8
+    need = lib.moe_ffn_w4a4_workspace_bytes(4, H, I, E, k)
+    tiles = lib.moe_w4a4_scale_tiles_bytes(H, I, E)
+    assert tiles == E * 3 * H * I // 16  # one E4M3 scale per 16 weights, re-laid out
+    call = lambda T, H, I, E, k, st=A, ws=A, wsb=need: lib.moe_grouped_ffn_w4a4(
+        A, ctypes.byref(r), ctypes.byref(ex), st, T, H, I, E, k, A, ws, wsb, None)
+    assert call(4, H, 1000, E, k) == SHAPE      # I % 128
+    assert call(4, 2176, I, E, k) == SHAPE      # H % 256
+    assert call(4, H, I, E, k, st=None) == INVALID  # the prepared weight-scale tiles are required
+    assert call(4, H, I, E, k, st=A + 8) == MISALIGNED
+    assert call(4, H, I, E, k, ws=None) == WS
+    assert call(4, H, I, E, k, wsb=need - 1) == WS
+    assert call(0, H, I, E, k, st=None, ws=None, wsb=0) == OK
+    ex.fmt = 0
+    assert call(4, H, I, E, k) == INVALID       # NVFP4 experts only
+    ex.fmt = 2
+    ex.w2_gscale = None
+    assert call(4, H, I, E, k) == INVALID       # per-expert scales required
+    prep = lambda H, I, E, out=A, nb=tiles: lib.moe_w4a4_prepare(ctypes.byref(ex), H, I, E, out, nb, None)
+    assert prep(H, I, E) == INVALID
+    ex.w2_gscale = A
+    assert prep(H, 1000, E) == SHAPE
+    assert prep(H, I, E, out=None) == INVALID
+    assert prep(H, I, E, nb=tiles - 1) == WS
+    assert prep(H, I, 2000) == SHAPE
+    # workspace: x and h quantised, routed x codes, h in fp32, tile-ordered activation scales
+    P = 4096 * 8
+    assert lib.moe_ffn_w4a4_workspace_bytes(4096, 7168, 2048, 256, 8) >= P * 2048 * 4 + P * 7168 // 2
 
 
 def test_select_bits_validation(lib):
