@@ -153,21 +153,26 @@ MOE_DEVICE void w4h_group(uint4 wa, uint4 wb, const uint4 (&xv)[2][4], float sa,
 // staged in the same pairing).  Plane p's register is bf16(2^(7-p)) in both halves with
 // the plane bit OR-ed into a mantissa or the sign bit, so A = 2^(7-p) (1 + g_j bit):
 //   j = 0..6   the bit stays in place (mantissa bit j):       g_j = 2^(j-7)
-//   j = 7..14  the bit moves to mantissa bit 6 (one shift):    g_j = 1/2
+//   j = 7..13  mantissa bit j-7 of w >> 7 (one shift per word): g_j = 2^(j-14)
+//   j = 14     the bit moves to mantissa bit 6 (one shift):    g_j = 1/2
 //   j = 15     the bit stays in place (the sign):              g_j = -2
 // With the activations staged as x'_k = x_k / g_j(k) (exact: powers of two), one
 // accumulator collects every plane:  T = sum_{p<b} 2^(7-p) (X' + sum_k bit_pk x_k),
 // X' = sum_k x'_k, so that, with X = sum_k x_k and u' the b-bit floor-and-compensation
 // code (floor = sum_{p<b} 2^(7-p) bit_p, compensation c_b = 2^(7-b) for b < 8, 0 for 8),
 //   sum_k (u'_k - 128) x_k = T - (256 - 2^(8-b)) X' + (c_b - 128) X.
+// w7 = w >> 7 (once per plane word): bits 7..13 sit in mantissa bits 0..6 of w7
 template <int J>
-MOE_DEVICE uint32_t bp_a(uint32_t w, uint32_t base) {
+MOE_DEVICE uint32_t bp_a(uint32_t w, uint32_t w7, uint32_t base) {
   if constexpr (J <= 6) return (w & (0x00010001u << J)) | base;
+  else if constexpr (J <= 13) return (w7 & (0x00010001u << (J - 7))) | base;
   else if constexpr (J == 15) return (w & 0x80008000u) | base;
   else return ((w >> (J - 6)) & 0x00400040u) | base;
 }
 // activation scale 1 / g_j of pair j
-MOE_DEVICE float bp_xscale(int j) { return j <= 6 ? float(1 << (7 - j)) : (j == 15 ? -0.5f : 2.f); }
+MOE_DEVICE float bp_xscale(int j) {
+  return j <= 6 ? float(1 << (7 - j)) : j <= 13 ? float(1 << (14 - j)) : (j == 15 ? -0.5f : 2.f);
+}
 
 // Widths of the chunk's tokens as one lane sees them: the C columns 2c, 2c+1 (+8) for
 // the epilogue, the B column g (+8) for the tail planes, and the chunk's min / max.
@@ -189,13 +194,14 @@ MOE_DEVICE void bp_plane(uint32_t wa, uint32_t wb, int p, const uint4 (&xv)[2][4
     keep[0] = p < bc.bB[0];
     keep[1] = p < bc.bB[1];
   }
+  const uint32_t wa7 = wa >> 7, wb7 = wb >> 7;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     uint32_t a0, a1, a2, a3;
-#define MOE_BP_STEP(S)                                         \
-  case S:                                                      \
-    a0 = bp_a<2 * S>(wa, base), a2 = bp_a<2 * S + 1>(wa, base); \
-    a1 = bp_a<2 * S>(wb, base), a3 = bp_a<2 * S + 1>(wb, base); \
+#define MOE_BP_STEP(S)                                                      \
+  case S:                                                                   \
+    a0 = bp_a<2 * S>(wa, wa7, base), a2 = bp_a<2 * S + 1>(wa, wa7, base); \
+    a1 = bp_a<2 * S>(wb, wb7, base), a3 = bp_a<2 * S + 1>(wb, wb7, base); \
     break;
     switch (s) {
       MOE_BP_STEP(0)
@@ -206,8 +212,8 @@ MOE_DEVICE void bp_plane(uint32_t wa, uint32_t wb, int p, const uint4 (&xv)[2][4
       MOE_BP_STEP(5)
       MOE_BP_STEP(6)
       default:
-        a0 = bp_a<14>(wa, base), a2 = bp_a<15>(wa, base);
-        a1 = bp_a<14>(wb, base), a3 = bp_a<15>(wb, base);
+        a0 = bp_a<14>(wa, wa7, base), a2 = bp_a<15>(wa, wa7, base);
+        a1 = bp_a<14>(wb, wb7, base), a3 = bp_a<15>(wb, wb7, base);
         break;
     }
 #undef MOE_BP_STEP
