@@ -296,7 +296,8 @@ MOE_DEVICE void fp4_group(uint4 wa, uint4 wb, uint32_t scA, uint32_t scB, const 
 // ---------------------------------------------------------------- one W4 unit
 // Streams the warp's W4 unit two groups per step: waits for groups G, G+1, computes them,
 // and refills their slots with groups G + kDepthW4, G + kDepthW4 + 1 (one commit group per
-// step).  Per-lane addresses are formed once.
+// step).  Per-lane addresses are formed once; the steps are unrolled over one turn of the
+// ring, so every slot offset is a constant.
 template <bool TWO, class Issue>
 MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* wscale, const uint8_t* xbuf,
                           const float* xsum, int GK, int g, int c, int nvalid, Issue&& issue, float (&acc)[2][4]) {
@@ -310,32 +311,38 @@ MOE_DEVICE void stream_w4(const FfnArgs& a, const uint8_t* wsm, const uint16_t* 
   const uint16_t* wsa = wscale + g * GK;
   const uint16_t* wsb = wscale + (g + 8) * GK;
   const uint8_t* wl = wsm + g * 64 + c * 16;
-  for (int G = 0; G < GK; G += 2) {
-    cp_async_wait_n<D / 2 - 1>();
-    __syncwarp();  // every lane's copies of groups G, G+1 have landed
+  // the ring is walked D groups at a time, so every slot offset is a constant
+  for (int G0 = 0; G0 < GK; G0 += D) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int GG = G + h;
-      if (GG < GK) {
-        uint4 xv[2][4];
-        float S[2][2];
+    for (int hp = 0; hp < D; hp += 2) {
+      const int G = G0 + hp;
+      if (G >= GK) break;
+      cp_async_wait_n<D / 2 - 1>();
+      __syncwarp();  // every lane's copies of groups G, G+1 have landed
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+      for (int h = 0; h < 2; ++h) {
+        const int GG = G + h;
+        if (GG < GK) {
+          uint4 xv[2][4];
+          float S[2][2];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr[nt] + GG * 256 + m * 64);
-          const float2 s2 = *reinterpret_cast<const float2*>(sr + GG * kMaxTok + 8 * nt);
-          S[nt][0] = s2.x;
-          S[nt][1] = s2.y;
+          for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr[nt] + GG * 256 + m * 64);
+            const float2 s2 = *reinterpret_cast<const float2*>(sr + GG * kMaxTok + 8 * nt);
+            S[nt][0] = s2.x;
+            S[nt][1] = s2.y;
+          }
+          const uint8_t* wr = wl + (hp + h) * 1024;
+          w4h_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
+                         bf16_bits_to_float(wsa[GG]), bf16_bits_to_float(wsb[GG]), S, acc);
         }
-        const uint8_t* wr = wl + (GG % D) * 1024;
-        w4h_group<TWO>(*reinterpret_cast<const uint4*>(wr), *reinterpret_cast<const uint4*>(wr + 8 * 64), xv,
-                       bf16_bits_to_float(wsa[GG]), bf16_bits_to_float(wsb[GG]), S, acc);
       }
+      __syncwarp();  // every lane is done with these slots before they are refilled
+      if (G + D < GK) issue(G + D, hp);
+      if (G + D + 1 < GK) issue(G + D + 1, hp + 1);
+      cp_async_commit();
     }
-    __syncwarp();  // every lane is done with these slots before they are refilled
-    if (G + D < GK) issue(G + D);
-    if (G + D + 1 < GK) issue(G + D + 1);
-    cp_async_commit();
   }
 }
 
@@ -348,10 +355,11 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, int slot, cons
                             const uint8_t* xbuf, const float* xsum, int GK, int g, int c, int nvalid,
                             const BpChunk& bc, Issue&& issue, float (&acc)[2][4]) {
   constexpr int NT = TWO ? 2 : 1;
+  int ring = 0;  // G % D
   for (int G = 0; G < GK; ++G) {
     cp_async_wait_n<D - 1>();
     __syncwarp();  // every lane's copies of group G have landed
-    const uint8_t* sl = wsm + (G % D) * slot;
+    const uint8_t* sl = wsm + ring * slot;
     uint4 xv[2][4];
     float X[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, X2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
@@ -383,8 +391,9 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, int slot, cons
                      xv, acc);
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
-    if (G + D < GK) issue(G + D);
+    if (G + D < GK) issue(G + D, ring);
     cp_async_commit();
+    ring = (ring == D - 1) ? 0 : ring + 1;
   }
 }
 
@@ -481,8 +490,8 @@ __global__ void __launch_bounds__(32 * WARPS, 16 / WARPS) k_ffn_gemv(FfnArgs a) 
     // ring geometry of this chunk: bitplane slots hold the chunk's nplanes planes only
     const int ring_slot = (FMT == MOE_FMT_BITPLANE8) ? nplanes * kRows * 16 : a.slot_bytes;
     const int ring_depth = (FMT == MOE_FMT_BITPLANE8) ? bp_depth(nplanes) : depth_of<FMT>();
-    auto issue = [&](int G) {  // copy group G of the unit into ring slot G % ring_depth
-      uint8_t* dst = wsm + (G % ring_depth) * ring_slot;
+    auto issue = [&](int G, int slot) {  // copy group G of the unit into ring slot `slot` (= G % ring_depth)
+      uint8_t* dst = wsm + slot * ring_slot;
       if (FMT == MOE_FMT_BITPLANE8) {
         const int i = lane & 15;
         for (int p = lane >> 4; p < nplanes; p += 2)
@@ -527,13 +536,13 @@ __global__ void __launch_bounds__(32 * WARPS, 16 / WARPS) k_ffn_gemv(FfnArgs a) 
       }
       if (FMT == MOE_FMT_W4G128) {  // two groups per commit group
         for (int G = 0; G < kDepthW4; G += 2) {
-          if (G < GK) issue(G);
-          if (G + 1 < GK) issue(G + 1);
+          if (G < GK) issue(G, G);
+          if (G + 1 < GK) issue(G + 1, G + 1);
           cp_async_commit();
         }
       } else {
         for (int G = 0; G < ring_depth; ++G) {
-          if (G < GK) issue(G);
+          if (G < GK) issue(G, G);
           cp_async_commit();
         }
       }
