@@ -355,8 +355,11 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, int slot, cons
                             const uint8_t* xbuf, const float* xsum, int GK, int g, int c, int nvalid,
                             const BpChunk& bc, Issue&& issue, float (&acc)[2][4]) {
   constexpr int NT = TWO ? 2 : 1;
-  int ring = 0;  // G % D
-  for (int G = 0; G < GK; ++G) {
+  // B column of an absent token: any staged row will do (each output column depends only on
+  // its own B column, and absent columns are never stored)
+  const uint8_t* xb[2] = {xbuf + size_t(min(g, nvalid - 1)) * a.x_stride + c * 16,
+                          xbuf + size_t(min(8 + g, nvalid - 1)) * a.x_stride + c * 16};
+  auto step = [&](int G, int ring) {  // group G in ring slot `ring`, then its refill
     cp_async_wait_n<D - 1>();
     __syncwarp();  // every lane's copies of group G have landed
     const uint8_t* sl = wsm + ring * slot;
@@ -364,10 +367,7 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, int slot, cons
     float X[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, X2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      // B column of an absent token: any staged row will do (each output column depends
-      // only on its own B column, and absent columns are never stored)
-      const int row = min(nt * 8 + g, nvalid - 1);
-      const uint8_t* xr = xbuf + size_t(row) * a.x_stride + G * 256 + c * 16;
+      const uint8_t* xr = xb[nt] + G * 256;
 #pragma unroll
       for (int m = 0; m < 4; ++m) xv[nt][m] = *reinterpret_cast<const uint4*>(xr + m * 64);
       if (FMT == MOE_FMT_BITPLANE8) {  // group sums X, X' of C columns 2c, 2c+1 ([G][kMaxTok] each)
@@ -393,7 +393,21 @@ MOE_DEVICE void stream_unit(const FfnArgs& a, const uint8_t* wsm, int slot, cons
     __syncwarp();  // every lane is done with this slot before it is refilled
     if (G + D < GK) issue(G + D, ring);
     cp_async_commit();
-    ring = (ring == D - 1) ? 0 : ring + 1;
+  };
+  if constexpr (FMT == MOE_FMT_NVFP4) {  // one turn of the ring at a time: constant slot offsets
+    for (int G0 = 0; G0 < GK; G0 += D) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        if (G0 + d >= GK) break;
+        step(G0 + d, d);
+      }
+    }
+  } else {  // bitplanes: D depends on the chunk's widths; the slot is kept as a counter
+    int ring = 0;  // G % D
+    for (int G = 0; G < GK; ++G) {
+      step(G, ring);
+      ring = (ring == D - 1) ? 0 : ring + 1;
+    }
   }
 }
 
