@@ -178,7 +178,7 @@ MOE_DEVICE float bp_xscale(int j) {
 // the epilogue, the B column g (+8) for the tail planes, and the chunk's min / max.
 struct BpChunk {
   int nplanes, pmin;
-  int bt[2][2];
+  float k1[2][2], k2[2][2];  // per C column: 256 - 2^(8-b) and c_b - 128 of its width b
   int bB[2];
 };
 
@@ -251,11 +251,7 @@ MOE_DEVICE void bp_group(const uint8_t* pl, const BpChunk& bc, const uint4 (&xv)
     if (nt == 1 && !TWO) break;
     float corr[2];
 #pragma unroll
-    for (int jj = 0; jj < 2; ++jj) {
-      const int b = bc.bt[nt][jj];
-      const float k1 = float(256 - (1 << (8 - b))), k2 = float((b < 8 ? (1 << (7 - b)) : 0) - 128);
-      corr[jj] = fmaf(k2, X[nt][jj], -k1 * X2[nt][jj]);
-    }
+    for (int jj = 0; jj < 2; ++jj) corr[jj] = fmaf(bc.k2[nt][jj], X[nt][jj], -bc.k1[nt][jj] * X2[nt][jj]);
     acc[nt][0] = fmaf(sa, (t0[nt][0] + t1[nt][0]) + corr[0], acc[nt][0]);
     acc[nt][1] = fmaf(sa, (t0[nt][1] + t1[nt][1]) + corr[1], acc[nt][1]);
     acc[nt][2] = fmaf(sb, (t0[nt][2] + t1[nt][2]) + corr[0], acc[nt][2]);
@@ -660,12 +656,16 @@ __global__ void __launch_bounds__(32 * WARPS, 16 / WARPS) k_ffn_gemv(FfnArgs a) 
     __syncthreads();
     if (!has_unit) continue;
 
-    BpChunk bc{nplanes, pmin, {{8, 8}, {8, 8}}, {8, 8}};
+    BpChunk bc{nplanes, pmin, {{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}, {8, 8}};
     if (FMT == MOE_FMT_BITPLANE8) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        bc.bt[nt][0] = sbits[nt * 8 + 2 * c];
-        bc.bt[nt][1] = sbits[nt * 8 + 2 * c + 1];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int b = sbits[nt * 8 + 2 * c + jj];
+          bc.k1[nt][jj] = float(256 - (1 << (8 - b)));
+          bc.k2[nt][jj] = float((b < 8 ? (1 << (7 - b)) : 0) - 128);
+        }
         bc.bB[nt] = sbits[nt * 8 + g];
       }
     }
