@@ -668,21 +668,30 @@ cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const 
 // byte kk.  The weight scales are laid out that way once per call from the row-major
 // scales (k_sf_tiles); the activation scales by their quantiser's row scatter.
 constexpr int kF4TM = 128, kF4TN = 128;
-constexpr int kF4Stages = 6;                        // K stages of 256 elements (128 bytes per row)
+constexpr int kF4Stages = 3;                        // K stages of 256 elements (128 bytes per row)
+// Two CTAs per SM, each with one accumulator buffer: one CTA's epilogue overlaps the other's
+// main loop (measured faster than one CTA with six stages and two accumulator buffers).
+constexpr int kF4AccBufs = 1;
+constexpr int kF4TmemCols = 256;                    // per CTA: two CTAs share the SM's 512 columns
 constexpr int kF4ABytes = kF4TM * 128, kF4BBytes = kF4TN * 128, kF4SfBytes = 4 * 512;
 constexpr int kF4StageBytes = kF4ABytes + kF4BBytes + 2 * kF4SfBytes;  // 36 KiB
 constexpr int kF4OffPre = kF4Stages * kF4StageBytes;
-constexpr int kF4OffOffs = kF4OffPre + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
-constexpr int kF4OffBar = kF4OffOffs + ((MOE_MAX_EXPERTS + 1) * 4 + 255) / 256 * 256;
 constexpr int kF4NumBars = 2 * kF4Stages + 4;
-constexpr int kF4OffTmemSlot = kF4OffBar + kF4NumBars * 8;
-constexpr int kF4SmemBytes = kF4OffTmemSlot + 16 + 1024;
+// shared memory after the stages: the row-tile prefix and the routing offsets ([E+1] each),
+// the barriers, the tensor-memory slot; + 1024 bytes of alignment slack.  E <= 256 keeps
+// two CTAs per SM (~112 KiB each); larger E runs one.
+__host__ __device__ constexpr int f4_offs_bytes(int E) { return ((E + 1) * 4 + 255) / 256 * 256; }
+__host__ __device__ constexpr int f4_smem_bytes(int E) {
+  return kF4OffPre + 2 * f4_offs_bytes(E) + kF4NumBars * 8 + 16 + 1024;
+}
+constexpr int kF4SmemMax = f4_smem_bytes(MOE_MAX_EXPERTS);
 constexpr int kF4Threads = 256;                     // producer, MMA, 2 idle, 4 epilogue warps
-// tensor-memory columns: accumulators at 0 and 128, the scales of stage s at 256 + 32 s (A)
-// and 272 + 32 s (B), 4 columns per 64-element K block
-constexpr uint32_t kF4SfaCol = 2 * kF4TN, kF4SfbCol = 2 * kF4TN + 16, kF4SfStageCols = 32;
-static_assert(kF4SfaCol + kF4Stages * kF4SfStageCols <= 512, "tensor-memory plan");
-static_assert(kF4SmemBytes <= 227 * 1024, "shared-memory plan");
+// tensor-memory columns: the accumulator at 0, the scales of stage s at 128 + 32 s (A) and
+// 144 + 32 s (B), 4 columns per 64-element K block
+constexpr uint32_t kF4SfaCol = kF4AccBufs * kF4TN, kF4SfbCol = kF4AccBufs * kF4TN + 16, kF4SfStageCols = 32;
+static_assert(kF4SfaCol + kF4Stages * kF4SfStageCols <= kF4TmemCols, "tensor-memory plan");
+static_assert(kF4SmemMax <= 227 * 1024, "shared-memory plan");
+static_assert(2 * f4_smem_bytes(256) + 2048 <= 228 * 1024, "two CTAs per SM at E <= 256");
 static_assert(kF4StageBytes % 1024 == 0, "stage alignment for the 128-byte swizzle");
 
 struct F4Args {
@@ -745,22 +754,22 @@ MOE_DEVICE Tile tile_of_n(int item, const int* pre, int E, int wtiles, const int
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kF4Threads, 1)
+__global__ void __launch_bounds__(kF4Threads, 2)
     k_ffn_fp4(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w, F4Args a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
+  const int E = a.E;
   int* pre = reinterpret_cast<int*>(smem + kF4OffPre);
-  int* offs = reinterpret_cast<int*>(smem + kF4OffOffs);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF4OffBar);
+  int* offs = reinterpret_cast<int*>(smem + kF4OffPre + f4_offs_bytes(E));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF4OffPre + 2 * f4_offs_bytes(E));
   uint64_t* full = bars;
   uint64_t* empty = full + kF4Stages;
   uint64_t* accFull = empty + kF4Stages;
   uint64_t* accEmpty = accFull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kF4OffTmemSlot);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kF4NumBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int E = a.E;
 
   for (int i = tid; i <= E; i += blockDim.x) offs[i] = a.offsets[i];
   __syncthreads();
@@ -792,7 +801,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     }
     fence_mbar_init();
   } else if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, kF4TmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -844,8 +853,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       int n = 0, it = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
-        const int ab = it & 1;
-        if (!mbar_wait(&accEmpty[ab], ((it >> 1) & 1) ^ 1, a.err)) break;
+        const int ab = it % kF4AccBufs;
+        if (!mbar_wait(&accEmpty[ab], ((it / kF4AccBufs) & 1) ^ 1, a.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + uint32_t(ab * kF4TN);
         for (int ks = 0; ks < KS; ++ks, ++n) {
@@ -875,7 +884,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         }
         if (ok) tc_commit(&accFull[ab]);
       }
-      if (it > 0 && ok) mbar_wait(&accFull[(it - 1) & 1], ((it - 1) >> 1) & 1, a.err);
+      if (it > 0 && ok) mbar_wait(&accFull[(it - 1) % kF4AccBufs], ((it - 1) / kF4AccBufs) & 1, a.err);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -886,8 +895,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
       int rt = 0;
       const Tile tl = tile_of_n(item, pre, E, a.wtiles, offs, kF4TN, &rt);
-      const int ab = it & 1;
-      if (!warp_wait(&accFull[ab], (it >> 1) & 1, a.err)) break;
+      const int ab = it % kF4AccBufs;
+      if (!warp_wait(&accFull[ab], (it / kF4AccBufs) & 1, a.err)) break;
       tc_fence_after();
       const float post = a.gs[tl.e] * __fdiv_rn(*a.act_amax, 2688.0f);
       float amax = 0.f;
@@ -928,7 +937,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kF4TmemCols);
   }
 }
 
@@ -1022,13 +1031,13 @@ cudaError_t launch_fp4_one(const CUtensorMap& tb, const CUtensorMap& tw, const F
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!raised[dev].load(std::memory_order_relaxed)) {
     const cudaError_t err = cudaFuncSetAttribute(k_ffn_fp4<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kF4SmemBytes);
+                                                 kF4SmemMax);
     if (err != cudaSuccess) return err;
     raised[dev].store(true, std::memory_order_relaxed);
   }
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  k_ffn_fp4<MODE><<<nsm, kF4Threads, kF4SmemBytes, st>>>(tb, tw, a);
+  k_ffn_fp4<MODE><<<2 * nsm, kF4Threads, f4_smem_bytes(a.E), st>>>(tb, tw, a);
   return cudaGetLastError();
 }
 

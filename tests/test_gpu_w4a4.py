@@ -48,6 +48,7 @@ W4A4_CASES = [
     (5, 1024, 512, 8, 2, False),     # decode-sized batch on the GEMM
     (300, 2048, 1024, 8, 2, False),  # OLMoE-like expert shape
     (512, 7168, 2048, 4, 2, False),  # the benchmark's expert shape: 28 K stages, 2 row tiles per expert
+    (64, 256, 128, 520, 2, False),   # E > 256: larger per-CTA tables, one CTA per SM; most experts empty
 ]
 
 
