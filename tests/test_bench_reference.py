@@ -62,3 +62,11 @@ def test_path_and_bytes_per_workload():
     # NVFP4: half a byte + one E4M3 byte per 16 weights + two fp32 per-tensor scales
     n = 3 * 7168 * 2048
     assert bench.expert_bytes(c["layer-h7168-e256-t1-nvfp4"]) == n // 2 + n // 16 + 8
+
+
+def test_w4a4_workload():
+    # NVFP4 weights and activations at the DeepSeek-like prefill shape: always the GEMM path,
+    # one record of its own in the default run
+    c = bench.LAYER_WORKLOADS["prefill-h7168-e256-w4a4"]
+    assert c.get("act") == "nvfp4" and c.get("fmt") == "nvfp4" and (c["H"], c["I"], c["E"], c["T"]) == (7168, 2048, 256, 4096)
+    assert bench.gemm_path(c) and "prefill-h7168-e256-w4a4" in bench.EXTRA_WORKLOADS
