@@ -172,6 +172,8 @@ FFN_CASES = [
     (3, 768, 384, 8, 2),       # K = 768 / 384: uneven split of groups over warps
     (90, 1024, 256, 4, 1),     # ~22 tokens per expert: two token chunks per weight pass
     (20, 7168, 384, 3, 1),     # K = 7168: seven weight stages per unit, 56 scale groups
+    (1, 2048, 1024, 64, 8),    # batch 1 (OLMoE-like): one token per expert
+    (2, 768, 384, 8, 2),       # batch 2; down K = 384 has an odd number of scale groups
 ]
 
 
