@@ -28,9 +28,14 @@
 //               per sub-partition overlap each other's waits; the fp16 weight operand
 //               never exists in shared memory;
 //   warps 12-15 drain one of the two accumulators (tcgen05.ld) while the other is
-//               being accumulated, apply SwiGLU, and store bf16 rows.
+//               being accumulated, apply SwiGLU, and store h (fp16, scaled) or y (bf16).
 // The work list (expert, row tile, weight tile) is built by every CTA from the
-// routing offsets and walked round-robin across CTAs.
+// routing offsets and walked round-robin across CTAs; experts with at most 16 routed
+// rows get no tiles and are left to a pass of the weight-streaming GEMV.
+//
+// The same file holds the W4A4 path (k_ffn_fp4 and its helpers, further down): NVFP4
+// weights and activations, both fed as E2M1 codes with E4M3 block scales to the
+// block-scaled FP4 MMA (kind::mxf4nvf4).
 //
 // Dequantisation (W4 group-128): (u - 8) * s with u the stored nibble and s the
 // group's bf16 scale, formed as fp16 (1024 + u) by byte permutes, then an fp16 add of
@@ -665,8 +670,9 @@ cudaError_t launch_umma_one(const CUtensorMap& tb, const CUtensorMap& tw, const 
 // K block (one MMA) a scale block of 512 bytes holds, for tile row m = m0 + 32 m1 and its
 // four 16-element sub-blocks kk, the byte 16 m0 + 4 m1 + kk; tcgen05.cp (32x128b, warpx4)
 // puts it into four tensor-memory columns of every lane quarter: lane 32 r + m0, column m1,
-// byte kk.  The weight scales are laid out that way once per call from the row-major
-// scales (k_sf_tiles); the activation scales by their quantiser's row scatter.
+// byte kk.  The weight scales are laid out that way once per set of experts from the
+// row-major scales (k_sf_tiles_w, moe_w4a4_prepare); the activation scales in every call by
+// the routed-row scatter (k_route_fp4_rows).
 constexpr int kF4TM = 128, kF4TN = 128;
 constexpr int kF4Stages = 3;                        // K stages of 256 elements (128 bytes per row)
 // Two CTAs per SM, each with one accumulator buffer: one CTA's epilogue overlaps the other's
