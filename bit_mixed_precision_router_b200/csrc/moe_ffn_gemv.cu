@@ -7,7 +7,9 @@
 //   down:    rows 0..15 = down rows 16t..16t+15.
 // One CTA = one routed expert x 4 warps, each warp owning one 16-row unit; four CTAs per
 // SM (small CTAs start at different times, so one CTA staging its tokens overlaps the
-// other CTAs' weight streams).  The expert's
+// other CTAs' weight streams).  Wide rows (K = 7168: one staged token row fits a 4-warp
+// CTA's budget) take one CTA of 16 warps per SM instead, whose stage holds several rows;
+// bitplanes use 8-warp CTAs, two per SM.  The expert's
 // activations for a chunk of up to `nx` tokens are staged once per CTA in shared memory,
 // already paired the way the dequantised weights pair them and with their per-group sums.
 // Each warp then streams its own units group by group (16 rows x 128 K-elements per group)
@@ -15,7 +17,9 @@
 // groups ahead (commit/wait groups, no cross-warp handshake), and per group: shared loads,
 // nibble / bit / FP4 -> fp16 or bf16 in registers, mma.sync m16n8k16 with the tokens on N.
 // W4 takes two groups per wait and converts nibbles to fp16 against activations staged
-// in fp16 (see w4h_group).  Expert weights are read from HBM once per token chunk.
+// in fp16 (see w4h_group); its group loop is unrolled over one turn of the ring, so slot
+// offsets are constants.  Expert weights are read from HBM once per token chunk.  In a
+// tensor-core GEMM batch the same kernel runs over the experts with at most 16 rows only.
 #include <atomic>
 #include <climits>
 
