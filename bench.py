@@ -241,10 +241,15 @@ def committed_traffic(name: str = "traffic.json"):
 
 
 def kernel_source_hash() -> str:
+    """Hash of the GEMV source's code (comment lines and blank lines left out), which keys
+    the committed DRAM-traffic records: they count only for the code they were taken on."""
     import hashlib
     h = hashlib.sha256()
     p = os.path.join(ROOT, "bit_mixed_precision_router_b200", "csrc", "moe_ffn_gemv.cu")
-    h.update(open(p, "rb").read())
+    for line in open(p, encoding="utf-8"):
+        t = line.strip()
+        if t and not t.startswith("//"):
+            h.update(t.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
