@@ -359,8 +359,9 @@ size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64
  * Two execution paths, chosen on the host from the shape alone (nothing is read back
  * from the device): with T*k >= 32*E and W4G128 or NVFP4 weights, a tensor-core GEMM
  * (weights dequantised into tensor memory once per tile of up to 192 routed rows, fp16
- * operands: W4 weights q*s, NVFP4 weights e2m1*e4m3); otherwise a weight-streaming GEMV
- * (dequantisation in registers, weights read once per pass of up to 16 rows).  For
+ * operands: W4 weights q*s, NVFP4 weights e2m1*e4m3) for the experts with more than 16
+ * routed rows, followed by the weight-streaming GEMV for the others; otherwise the GEMV
+ * alone (dequantisation in registers, weights read once per pass of up to 16 rows).  For
  * BITPLANE8 expert e is read at bits[p] planes for pair p (planes 0..bits[p]-1, floor
  * and compensation as above); expert e's weights are fetched to max_p bits[p].
  *   x bf16 [T][H];  routing: as written by moe_route_topk;  bits uint8 [T*k]
@@ -369,7 +370,7 @@ size_t moe_ffn_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64
  * >= moe_ffn_workspace_bytes(...) (scratch: h, and for the GEMM path the token rows
  * gathered into routed order; contents need not be initialised).  Not bit-exact: fp32
  * accumulation order, the rounding of h (and, on the GEMM path, of each dequantised
- * W4 weight to bf16) differ from an fp64 reference (ExactMoE: the low-bit layer is
+ * W4 weight to fp16) differ from an fp64 reference (ExactMoE: the low-bit layer is
  * not numerically identical to BF16); the FFN tolerance covers both paths.
  * Range: the W4 paths stage activations as fp16 x/16 and x/256 (GEMV) or x/16 and h/16
  * (GEMM), the NVFP4 paths activations and h as fp16 * 2^-8, so |x|, |h| < 2^20 (W4) and
