@@ -222,3 +222,47 @@ def test_device_cache_validation(lib):
     assert perm(4, 2, 8, ids=None) == INVALID
     assert perm(4, 2, 8, ids=A + 4) == MISALIGNED
     assert perm(0, 2, 8) == OK
+
+
+def test_remaining_entry_points_validation(lib):
+    # activation quantiser (fp32 rows, NVFP4 codes): 16-wide blocks, every pointer required
+    q = lambda R, C, a=A, sc=A: lib.moe_quantize_nvfp4_f32(a, R, C, A, sc, A, None)
+    assert q(4, 40) == SHAPE
+    assert q(0, 64) == INVALID
+    assert q(4, 64, a=None) == INVALID
+    assert q(4, 64, sc=None) == INVALID
+    assert q(4, 64, a=A + 4) == MISALIGNED
+    # the no-alloc router: shape limits of its fixed array, then pointers
+    r = _routing()
+    na = lambda T, H, E, k, x=A: lib.moe_route_topk_noalloc(x, A, None, T, H, E, k, ctypes.byref(r), None)
+    assert na(-1, 256, 8, 2) == INVALID
+    assert na(4, 200, 8, 2) == SHAPE
+    assert na(4, 256, 8, 9) == SHAPE
+    assert na(65536 // 64 + 1, 256, 64, 8) == SHAPE   # T * E above MOE_NOALLOC_MAX_LOGITS
+    assert na(0, 256, 8, 2, x=None) == OK             # no tokens: nothing to do, nothing looked up
+    assert na(4, 256, 8, 2, x=None) == INVALID
+    r.expert_list = None
+    assert na(4, 256, 8, 2) == INVALID
+    r.expert_list = A + 8
+    assert na(4, 256, 8, 2) == MISALIGNED
+    r.expert_list = A
+    assert na(4, 256, 8, 2, x=A + 2) == MISALIGNED
+    # expert parallelism: row gather and local ids from the exchanged counts
+    g = lambda n, div, H, src=A, idx=A: lib.moe_gather_rows(src, idx, n, div, H, A, None)
+    assert g(-1, 1, 2048) == INVALID
+    assert g(4, 0, 2048) == INVALID
+    assert g(4, 1, 2044) == SHAPE
+    assert g(0, 1, 2048, src=None) == OK
+    assert g(4, 1, 2048, idx=None) == INVALID
+    assert g(4, 1, 2048, src=A + 8) == MISALIGNED
+    assert g(4, 1, 2048, idx=A + 2) == MISALIGNED
+    c = lambda S, El, counts=A: lib.moe_ids_from_counts(counts, S, El, A, None)
+    assert c(0, 8) == INVALID
+    assert c(2, 0) == INVALID
+    assert c(2, 8, counts=None) == INVALID
+    assert c(1 << 11, 1 << 10) == SHAPE
+    assert c(2, 8, counts=A + 2) == MISALIGNED
+    # seeded generator
+    assert lib.moe_synth_uniform_bf16(None, 4, 0, 1, -1.0, 1.0, None) == INVALID
+    assert lib.moe_synth_uniform_bf16(A, 4, -1, 1, -1.0, 1.0, None) == INVALID
+    assert lib.moe_synth_uniform_bf16(A, 0, 0, 1, -1.0, 1.0, None) == OK
