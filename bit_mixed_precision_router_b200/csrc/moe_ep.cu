@@ -54,9 +54,9 @@ __global__ void __launch_bounds__(1024) k_ids_from_counts(const int32_t* __restr
 cudaError_t launch_gather_rows_by(const uint16_t* src, const int32_t* idx, int n, int div, int H, uint16_t* dst,
                                   cudaStream_t st) {
   const int threads = 256;
-  int blocks = (n * 32 + threads - 1) / threads;
+  int64_t blocks = (int64_t(n) * 32 + threads - 1) / threads;
   blocks = blocks < 1 ? 1 : (blocks > 4096 ? 4096 : blocks);
-  k_gather_rows_by<<<blocks, threads, 0, st>>>(reinterpret_cast<const uint4*>(src), idx, n, div, H / 8,
+  k_gather_rows_by<<<unsigned(blocks), threads, 0, st>>>(reinterpret_cast<const uint4*>(src), idx, n, div, H / 8,
                                                reinterpret_cast<uint4*>(dst));
   return cudaGetLastError();
 }
