@@ -70,3 +70,20 @@ def test_w4a4_workload():
     c = bench.LAYER_WORKLOADS["prefill-h7168-e256-w4a4"]
     assert c.get("act") == "nvfp4" and c.get("fmt") == "nvfp4" and (c["H"], c["I"], c["E"], c["T"]) == (7168, 2048, 256, 4096)
     assert bench.gemm_path(c) and "prefill-h7168-e256-w4a4" in bench.EXTRA_WORKLOADS
+
+
+def test_profile_commands_run_the_current_bench():
+    # every bench.py command line quoted in profiles/ parses with the current flags, so each
+    # committed summary can be re-made from committed files
+    import glob
+    import os
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    n = 0
+    for f in sorted(glob.glob(os.path.join(root, "profiles", "*.md"))):
+        text = open(f).read().replace("\\\n", " ")
+        assert "--clock-control none" in text, f
+        for m in re.finditer(r"python bench\.py([^>&\n`'\";|]*)", text):
+            bench.parse_args(m.group(1).split())
+            n += 1
+    assert n >= 8
